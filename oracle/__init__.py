@@ -1,0 +1,30 @@
+"""CPU fp64 oracle for the online-softmax attention forward.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call, link or
+execute anything in this package: only ``tests/``, ``__graft_entry__.smoke()``
+and ``bench.py``'s ``cpu_baseline`` leg (and its ``--impl reference`` arm) use
+it. The oracle shares no code with the CUDA library: it reads the same stored
+input bits (bf16, fp32, e4m3fn bytes) and evaluates the plain definition
+
+    out = softmax(softmax_scale * Q K^T + additive_mask) V
+
+in float64, two passes per query row (row max, then exp / sum / P V).
+
+Modules
+-------
+attention   -- the definition for the three entry points (encoder, GQA decode,
+               paged history) plus the split-KV log-sum-exp combine.
+e4m3        -- an FP8 E4M3FN decoder written from the format definition.
+flops       -- the closed-form work counts used for throughput figures.
+"""
+
+from .attention import (  # noqa: F401
+    softmax_attention,
+    encoder_attention,
+    gqa_decode_attention,
+    paged_history_attention,
+    paged_logical_kv,
+    lse_combine,
+)
+from .e4m3 import e4m3fn_to_float64  # noqa: F401
+from .flops import attention_flops, decode_algorithmic_bytes  # noqa: F401
