@@ -1,0 +1,170 @@
+/*
+ * attn.h -- C ABI of libattn_b200.so, the B200 (sm_100a) online-softmax
+ * ("flash") attention forward:
+ *
+ *     out = softmax(softmax_scale * Q K^T + additive_mask) V
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never frees them and never keeps them after the call returns. The library
+ *    allocates no device memory: besides the caller's buffers it only uses one
+ *    per-device status word (a static __device__ variable) and kernel
+ *    parameters.
+ *  - bf16 tensors are passed as `const uint16_t*` holding bf16 bit patterns
+ *    (1 sign, 8 exponent, 7 mantissa bits). FP8 caches are `const uint8_t*`
+ *    holding E4M3FN codes. All tensors are dense, row-major, contiguous in the
+ *    layouts stated per function, and every tensor base address must be
+ *    16-byte aligned (it is read by the Tensor Memory Accelerator).
+ *  - `stream` is a `cudaStream_t` passed as `void*` (NULL = legacy default
+ *    stream). Every function only validates its arguments on the host and
+ *    enqueues work: it returns before the GPU has finished.
+ *  - Return value: ATTN_OK or a negative attn_status. A host-side validation
+ *    failure enqueues nothing. Errors the device detects (an out-of-range block
+ *    table entry, a bounded wait that ran out) are recorded in the per-device
+ *    status word and reported by attn_check().
+ *  - softmax_scale must be finite and > 0. Rows whose every key is masked
+ *    produce an all-zero output row.
+ *  - Nothing here falls back to another implementation: an unsupported shape
+ *    is an error.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_status {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,           /* a required pointer is NULL                      */
+    ATTN_ERR_SHAPE = -2,          /* inconsistent or out-of-range sizes / scale      */
+    ATTN_ERR_UNSUPPORTED = -3,    /* valid attention, but a shape this build rejects */
+    ATTN_ERR_ALIGN = -4,          /* a base address is not 16-byte aligned           */
+    ATTN_ERR_WORKSPACE = -5,      /* workspace missing or too small                  */
+    ATTN_ERR_CUDA = -6,           /* a CUDA runtime / driver call failed             */
+    ATTN_ERR_DEVICE_TIMEOUT = -7, /* a kernel's bounded wait ran out (device side)   */
+    ATTN_ERR_BLOCK_TABLE = -8     /* a block-table entry is outside the pool (device)*/
+} attn_status;
+
+/*
+ * attn_encoder_fwd -- non-causal multi-head encoder attention.
+ *
+ * Defined by: "V-JEPA2 ViT-L Encoder NKI Kernels for AWS Trainium2" (the K2
+ * attention inner, "Repository layout"), "vit-encoder-neuron-kernels"
+ * ("Supported shapes and limits": bidirectional self-attention, head_dim 64 or
+ * 128) and "gte-encoder-neuron-kernels" ("Constraints": right padding with a
+ * 0/1 attention_mask, here generalised to an additive per-key bias).
+ *
+ *   q, k, v, out : [B, H, S, D] bf16. out may not alias q, k or v.
+ *   B, H >= 1; S >= 1; D in {64, 128}.
+ *   softmax_scale: finite, > 0 (1/sqrt(D) for the ViT encoders).
+ *   key_bias     : NULL, or [B, S] fp32 additive bias added to every query's
+ *                  score for key j of batch entry b (0 keep, -inf drop).
+ *
+ * Every query row attends to all S keys (no causal mask). Accumulation is fp32;
+ * out is rounded to bf16 (round-to-nearest-even).
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_ALIGN,
+ * ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_encoder_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                     int B, int H, int S, int D, float softmax_scale,
+                     const float* key_bias, void* stream);
+
+/*
+ * attn_gqa_decode_workspace_size -- bytes of device workspace attn_gqa_decode
+ * needs for these sizes (the split-KV partial results). 0 for invalid sizes.
+ */
+ATTN_API size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx, int D);
+
+/*
+ * attn_gqa_decode -- single-token (S_q = 1) GQA flash-decode.
+ *
+ * Defined by: "head_dim>128 (256/512) GQA Flash-Decode NKI Kernel for AWS
+ * Trainium", sections "Input contract" and "Supported shapes (the eligibility
+ * gate)"; the key-sequence split with a log-sum-exp combine is the page's
+ * "Future performance follow-on" (multi-program dispatch).
+ *
+ *   q         : [B, Hq, 1, D] bf16
+ *   k, v      : [B, Hkv, S_ctx, D] bf16
+ *   attn_mask : NULL (no mask), or [B, 1, 1, S_ctx] fp32 additive (0 keep,
+ *               -inf drop). A -inf entry removes the key whatever its K holds.
+ *   out       : [B, Hq, 1, D] bf16
+ *   Hq == Hkv * num_kv_groups; query head h reads kv head h / num_kv_groups.
+ *   D in {128, 256, 512}; S_ctx >= 1 (no multiple-of-128 requirement).
+ *   workspace : device buffer of at least attn_gqa_decode_workspace_size(...)
+ *               bytes, 16-byte aligned, owned by the caller; its contents on
+ *               entry do not matter. Calls that share one workspace must not
+ *               overlap on the GPU.
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_ALIGN,
+ * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                    const float* attn_mask, uint16_t* out,
+                    int B, int Hq, int Hkv, int num_kv_groups, int S_ctx, int D,
+                    float softmax_scale, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
+ * attn_paged_history -- history-only attention over a paged FP8 KV cache.
+ *
+ * Defined by: "Prefill Context-Parallel Attention POC for Trainium2",
+ * sections "Layout" (Q [Hq, q_len, D], K/V [blocks, Hkv, block_size, D],
+ * O [Hq, q_len, D]), the history-only rule under the target configuration,
+ * the runtime additive bias from actual_history_len, and "Current POC
+ * constraints" (head_dim multiple of 128, block_size <= 512 and a multiple of
+ * 128, Q bf16, K/V FP8 E4M3FN, fp32 max/sum). On one GPU the page's ring of
+ * ranks becomes a loop over the blocks named by the block table.
+ *
+ *   q            : [Hq, Sq, D] bf16
+ *   k_cache      : [num_phys_blocks, Hkv, block_size, D] E4M3FN codes
+ *   v_cache      : same layout as k_cache
+ *   block_table  : [n_table] int32, logical block i -> physical block
+ *                  block_table[i]; logical position t lives in logical block
+ *                  t / block_size at offset t % block_size.
+ *   actual_history_len : 0 <= len <= n_table * block_size. Positions >= len
+ *                  are ignored (a partial last block is allowed); blocks
+ *                  wholly beyond len are never read.
+ *   k_scale, v_scale   : per-tensor dequantisation scales (value = code * scale)
+ *   out          : [Hq, Sq, D] bf16
+ *   Hq == Hkv * num_kv_groups; D == 256; block_size in {128, 256, 384, 512}.
+ *   Every query attends to every history position < len (no causal mask).
+ * Table entries are checked on the device: an entry outside
+ * [0, num_phys_blocks) is skipped and recorded as ATTN_ERR_BLOCK_TABLE.
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_ALIGN,
+ * ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                       const int32_t* block_table, int n_table, int num_phys_blocks,
+                       int block_size, int actual_history_len,
+                       float k_scale, float v_scale, float softmax_scale,
+                       int Hq, int Hkv, int num_kv_groups, int Sq, int D,
+                       uint16_t* out, void* stream);
+
+/*
+ * attn_check -- synchronise `stream`, then return and clear the first error the
+ * device recorded on the current device since the last check (ATTN_OK if
+ * none). Returns ATTN_ERR_CUDA if the synchronisation itself fails.
+ */
+ATTN_API int attn_check(void* stream);
+
+/* attn_status_string -- static, human-readable name of a status code. */
+ATTN_API const char* attn_status_string(int status);
+
+/* attn_version -- library ABI version (major * 10000 + minor * 100 + patch). */
+ATTN_API int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

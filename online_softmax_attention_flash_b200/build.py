@@ -1,0 +1,63 @@
+"""Build libattn_b200.so in-tree with nvcc for sm_100a.
+
+    python -m online_softmax_attention_flash_b200.build [--verbose-ptxas]
+
+The library is one CUDA translation unit (csrc/attn_lib.cu) linked against the
+static CUDA runtime; it needs no GPU to build.
+"""
+
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG_DIR)
+CSRC = os.path.join(PKG_DIR, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB_NAME = "libattn_b200.so"
+LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
+ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc_path() -> str:
+    for cand in (shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def sources():
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)
+                  if f.endswith((".cu", ".cuh")))
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB_PATH):
+        return False
+    t = os.path.getmtime(LIB_PATH)
+    deps = sources() + [os.path.join(INCLUDE, "attn.h"), os.path.abspath(__file__)]
+    return all(os.path.getmtime(p) <= t for p in deps)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = LIB_PATH,
+          extra_flags=None) -> str:
+    if not force and out == LIB_PATH and up_to_date():
+        return out
+    cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
+           "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+           "-I", INCLUDE, "-I", CSRC,
+           "-o", out, os.path.join(CSRC, "attn_lib.cu")]
+    if verbose_ptxas:
+        cmd[1:1] = ["-Xptxas", "-v"]
+    if extra_flags:
+        cmd[1:1] = list(extra_flags)
+    subprocess.run(cmd, check=True)
+    return out
+
+
+if __name__ == "__main__":
+    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
+    print(LIB_PATH)

@@ -1,0 +1,201 @@
+// attn_lib.cu -- the C ABI of libattn_b200.so (declared in include/attn.h).
+//
+// One translation unit: the kernels are header-only (encoder.cuh, decode.cuh,
+// paged.cuh) and included here, so the per-device status word is a single
+// static __device__ variable. Host code validates arguments, encodes TMA
+// tensor maps, and launches on the caller's stream. It allocates nothing.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "decode.cuh"
+#include "encoder.cuh"
+#include "paged.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+// ------------------------------------------------------------ driver entry
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::once_flag g_encode_once;
+
+bool load_encode_tiled() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode_tiled != nullptr;
+}
+
+// Tiled map over a rank-3 row-major tensor [d2][d1][d0] with a 128-byte swizzle.
+// elem_bytes * box0 must be 128 (one swizzle row).
+int encode_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t elem_bytes,
+                  const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                  uint32_t box1) {
+    if (!load_encode_tiled()) return ATTN_ERR_CUDA;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode_tiled(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+
+// Dynamic shared memory opt-in, once per (kernel, device).
+template <typename K>
+int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done_mask.load(std::memory_order_acquire) & bit) return ATTN_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
+    done_mask.fetch_or(bit, std::memory_order_acq_rel);
+    return ATTN_OK;
+}
+
+template <int D, bool kBias>
+int launch_encoder(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
+                   int H, int S, float scale, const float* key_bias, cudaStream_t stream) {
+    using namespace attn::enc;
+    static std::atomic<uint64_t> smem_done{0};
+    auto kernel = encoder_fwd_kernel<D, kBias>;
+    int rc = ensure_smem(kernel, Cfg<D>::kSmemBytes, smem_done);
+    if (rc) return rc;
+    CUtensorMap tq, tk, tv;
+    const uint64_t rows = static_cast<uint64_t>(S);
+    const uint64_t heads = static_cast<uint64_t>(B) * H;
+    if ((rc = encode_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, D, rows, heads, 64, kTileM)))
+        return rc;
+    if ((rc = encode_map_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, D, rows, heads, 64, kTileN)))
+        return rc;
+    if ((rc = encode_map_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, D, rows, heads, 64, kTileN)))
+        return rc;
+    dim3 grid((S + kRowsPerCta - 1) / kRowsPerCta, static_cast<unsigned>(heads));
+    const float scale_log2 = scale * kLog2e;
+    kernel<<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, out, key_bias, H, S,
+                                                           scale_log2);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_version(void) { return kVersion; }
+
+const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_NULL: return "ATTN_ERR_NULL";
+        case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+        case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN";
+        case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT";
+        case ATTN_ERR_BLOCK_TABLE: return "ATTN_ERR_BLOCK_TABLE";
+        default: return "ATTN_ERR_UNKNOWN";
+    }
+}
+
+int attn_check(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, attn::g_attn_device_status, sizeof(int)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(attn::g_attn_device_status, &zero, sizeof(int)) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+    }
+    return v;
+}
+
+int attn_encoder_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                     int B, int H, int S, int D, float softmax_scale, const float* key_bias,
+                     void* stream) {
+    if (!q || !k || !v || !out) return ATTN_ERR_NULL;
+    if (B < 1 || H < 1 || S < 1 || !scale_ok(softmax_scale)) return ATTN_ERR_SHAPE;
+    if (static_cast<int64_t>(B) * H > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_ALIGN;
+    if (key_bias && (reinterpret_cast<uintptr_t>(key_bias) & 3u)) return ATTN_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (D == 64)
+        return key_bias ? launch_encoder<64, true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
+                        : launch_encoder<64, false>(q, k, v, out, B, H, S, softmax_scale, nullptr, st);
+    return key_bias ? launch_encoder<128, true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
+                    : launch_encoder<128, false>(q, k, v, out, B, H, S, softmax_scale, nullptr, st);
+}
+
+size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx, int D) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || S_ctx < 1 || D < 1 || Hq % Hkv) return 0;
+    return attn::dec::workspace_bytes(B, Hq, S_ctx, D);
+}
+
+int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                    const float* attn_mask, uint16_t* out, int B, int Hq, int Hkv,
+                    int num_kv_groups, int S_ctx, int D, float softmax_scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !out) return ATTN_ERR_NULL;
+    if (B < 1 || Hq < 1 || Hkv < 1 || S_ctx < 1 || num_kv_groups < 1) return ATTN_ERR_SHAPE;
+    if (Hq != Hkv * num_kv_groups || !scale_ok(softmax_scale)) return ATTN_ERR_SHAPE;
+    if (D != 128 && D != 256 && D != 512) return ATTN_ERR_UNSUPPORTED;
+    if (num_kv_groups > attn::dec::kMaxGroups) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_ALIGN;
+    if (attn_mask && (reinterpret_cast<uintptr_t>(attn_mask) & 15u)) return ATTN_ERR_ALIGN;
+    const size_t need = attn::dec::workspace_bytes(B, Hq, S_ctx, D);
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
+    return attn::dec::launch(q, k, v, attn_mask, out, B, Hq, Hkv, num_kv_groups, S_ctx, D,
+                             softmax_scale, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                       const int32_t* block_table, int n_table, int num_phys_blocks,
+                       int block_size, int actual_history_len, float k_scale, float v_scale,
+                       float softmax_scale, int Hq, int Hkv, int num_kv_groups, int Sq, int D,
+                       uint16_t* out, void* stream) {
+    if (!q || !k_cache || !v_cache || !block_table || !out) return ATTN_ERR_NULL;
+    if (Hq < 1 || Hkv < 1 || num_kv_groups < 1 || Hq != Hkv * num_kv_groups || Sq < 1)
+        return ATTN_ERR_SHAPE;
+    if (n_table < 0 || num_phys_blocks < 1 || actual_history_len < 0) return ATTN_ERR_SHAPE;
+    if (block_size < 128 || block_size > 512 || block_size % 128) return ATTN_ERR_SHAPE;
+    if (static_cast<int64_t>(actual_history_len) > static_cast<int64_t>(n_table) * block_size)
+        return ATTN_ERR_SHAPE;
+    if (!scale_ok(softmax_scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return ATTN_ERR_SHAPE;
+    if (D != 256) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u))
+        return ATTN_ERR_ALIGN;
+    return attn::paged::launch(q, k_cache, v_cache, block_table, n_table, num_phys_blocks,
+                               block_size, actual_history_len, k_scale, v_scale, softmax_scale,
+                               Hq, Hkv, num_kv_groups, Sq, D, out,
+                               static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+"""GPU parity of attn_gqa_decode against the fp64 oracle (through the C ABI)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from online_softmax_attention_flash_b200 import binding as B
+from online_softmax_attention_flash_b200 import inputs as syn
+from parity import assert_bf16_parity, to_f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _run(case: syn.DecodeCase, use_mask=True):
+    q, k, v = (t.to(DEV) for t in (case.q, case.k, case.v))
+    m = case.attn_mask.to(DEV) if (use_mask and case.attn_mask is not None) else None
+    out = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups)
+    assert B.attn_check() == 0
+    return out
+
+
+def _oracle(case: syn.DecodeCase, use_mask=True):
+    m = case.attn_mask.double().numpy() if (use_mask and case.attn_mask is not None) else None
+    return oracle.gqa_decode_attention(to_f64(case.q), to_f64(case.k), to_f64(case.v), m,
+                                       case.softmax_scale, case.num_kv_groups)
+
+
+def test_full_config_b8_16q_8kv_d256_ctx4096():
+    case = syn.gqa_decode_full_case()
+    assert_bf16_parity(_run(case), _oracle(case), 2, "decode full")
+
+
+@pytest.mark.parametrize("D", [128, 256, 512])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_head_dims_and_groups(D, G):
+    Hkv = 2
+    case = syn.decode_case(3, Hkv * G, Hkv, 700, D, seed=10 * D + G, softmax_scale=D ** -0.5,
+                           min_len=1, max_len=700)
+    assert_bf16_parity(_run(case), _oracle(case), 2, f"D={D} G={G}")
+
+
+@pytest.mark.parametrize("S_ctx", [1, 31, 32, 33, 255, 256, 257, 1000])
+def test_ragged_context_without_mask(S_ctx):
+    case = syn.decode_case(2, 4, 2, S_ctx, 256, seed=S_ctx, lengths=[S_ctx, S_ctx])
+    assert_bf16_parity(_run(case, use_mask=False), _oracle(case, use_mask=False), 2,
+                       f"S_ctx={S_ctx}")
+
+
+def test_random_neg_inf_pattern_and_finite_mask_values():
+    case = syn.decode_case(2, 4, 2, 1500, 256, seed=5)
+    g = torch.Generator().manual_seed(1)
+    m = torch.randn(2, 1, 1, 1500, generator=g)
+    m[torch.rand(2, 1, 1, 1500, generator=g) < 0.7] = float("-inf")
+    m[0, ..., 256:512] = float("-inf")          # one whole split removed
+    case.attn_mask = m
+    assert_bf16_parity(_run(case), _oracle(case), 2, "random mask")
+
+
+def test_single_unmasked_key_is_bit_exact():
+    case = syn.decode_case(2, 4, 2, 900, 256, seed=6)
+    case.attn_mask.fill_(float("-inf"))
+    case.attn_mask[0, ..., 0] = 0.0
+    case.attn_mask[1, ..., 777] = 2.5
+    out = _run(case).cpu()
+    for h in range(4):
+        assert torch.equal(out[0, h, 0], case.v[0, h // 2, 0])
+        assert torch.equal(out[1, h, 0], case.v[1, h // 2, 777])
+
+
+def test_masked_tail_equals_truncated_problem_bitwise():
+    L = 1337
+    full = syn.decode_case(2, 4, 2, 4096, 256, seed=7, lengths=[L, L])
+    trunc = syn.DecodeCase(full.q, full.k[:, :, :L].contiguous(), full.v[:, :, :L].contiguous(),
+                           None, full.lengths, full.softmax_scale, full.num_kv_groups)
+    a = _run(full).cpu()
+    b = _run(trunc, use_mask=False).cpu()
+    assert torch.equal(a, b)
+
+
+def test_gqa_equals_repeated_kv_heads():
+    case = syn.decode_case(2, 8, 2, 600, 256, seed=8)
+    rep = syn.DecodeCase(case.q, case.k.repeat_interleave(4, dim=1),
+                         case.v.repeat_interleave(4, dim=1), case.attn_mask, case.lengths,
+                         case.softmax_scale, 1)
+    assert torch.equal(_run(case).cpu(), _run(rep).cpu())
+
+
+def test_fully_masked_row_is_zero():
+    case = syn.decode_case(1, 2, 1, 300, 256, seed=9)
+    case.attn_mask.fill_(float("-inf"))
+    out = _run(case).cpu()
+    assert torch.count_nonzero(out) == 0

@@ -1,0 +1,106 @@
+"""GPU parity of attn_encoder_fwd against the fp64 oracle (through the C ABI)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from online_softmax_attention_flash_b200 import binding as B
+from online_softmax_attention_flash_b200 import inputs as syn
+from parity import assert_bf16_parity, to_f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _run(case: syn.EncoderCase):
+    q, k, v = (t.to(DEV) for t in (case.q, case.k, case.v))
+    kb = None if case.key_bias is None else case.key_bias.to(DEV)
+    out = B.attn_encoder_fwd(q, k, v, case.softmax_scale, key_bias=kb)
+    assert B.attn_check() == 0
+    return out
+
+
+def _oracle(case: syn.EncoderCase, rows=None):
+    kb = None if case.key_bias is None else case.key_bias.double().numpy()
+    return oracle.encoder_attention(to_f64(case.q), to_f64(case.k), to_f64(case.v),
+                                    case.softmax_scale, key_bias=kb, rows=rows)
+
+
+def test_tiny_mha_b1_h4_s256_d64():
+    case = syn.tiny_case()
+    assert_bf16_parity(_run(case), _oracle(case), 2, "tiny")
+
+
+def test_dinov3_b8_h16_s201_d64_ragged_tail():
+    case = syn.dinov3_case()
+    assert_bf16_parity(_run(case), _oracle(case), 2, "dinov3")
+
+
+@pytest.mark.parametrize("layer", [0, 23])
+def test_vitl_b1_h16_s2048_d64(layer):
+    case = syn.vitl_layer_case(layer)
+    assert_bf16_parity(_run(case), _oracle(case), 2, f"vitl layer {layer}")
+
+
+@pytest.mark.parametrize("S", [1, 7, 64, 127, 128, 129, 255, 256, 257, 300, 513])
+@pytest.mark.parametrize("D", [64, 128])
+def test_ragged_lengths(S, D):
+    case = syn.encoder_case(2, 3, S, D, seed=300 + S + D, softmax_scale=D ** -0.5)
+    assert_bf16_parity(_run(case), _oracle(case), 2, f"S={S} D={D}")
+
+
+def test_head_dim_128_long():
+    case = syn.encoder_case(1, 4, 1024, 128, seed=77, softmax_scale=128 ** -0.5)
+    assert_bf16_parity(_run(case), _oracle(case), 2, "D=128 S=1024")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_right_padding_key_bias(D):
+    case = syn.encoder_case(4, 2, 384, D, seed=91, softmax_scale=0.125,
+                            pad_lengths=[384, 200, 129, 6])
+    assert_bf16_parity(_run(case), _oracle(case), 2, "padding")
+
+
+def test_random_finite_key_bias():
+    case = syn.encoder_case(2, 2, 300, 64, seed=92)
+    g = torch.Generator().manual_seed(5)
+    case.key_bias = torch.randn(2, 300, generator=g) * 3.0
+    assert_bf16_parity(_run(case), _oracle(case), 2, "finite bias")
+
+
+def test_single_unmasked_key_is_bit_exact():
+    case = syn.encoder_case(2, 2, 200, 64, seed=93, pad_lengths=[1, 1])
+    case.key_bias[1, 0] = float("-inf")
+    case.key_bias[1, 137] = 0.0
+    out = _run(case).cpu()
+    assert torch.equal(out[0], case.v[0, :, 0:1].expand(2, 200, 64))
+    assert torch.equal(out[1], case.v[1, :, 137:138].expand(2, 200, 64))
+
+
+def test_fully_masked_rows_are_zero():
+    case = syn.encoder_case(1, 1, 140, 64, seed=94, pad_lengths=[0])
+    out = _run(case).cpu()
+    assert torch.count_nonzero(out) == 0
+
+
+def test_zero_query_gives_mean_of_values():
+    case = syn.encoder_case(1, 2, 333, 64, seed=95)
+    case.q.zero_()
+    ref = _oracle(case)
+    assert np.allclose(ref[0, :, 0], to_f64(case.v)[0].mean(axis=1))
+    assert_bf16_parity(_run(case), ref, 2, "q=0")
+
+
+def test_batch_independence_bitwise():
+    a = syn.encoder_case(2, 2, 201, 64, seed=96)
+    b = syn.encoder_case(2, 2, 201, 64, seed=97)
+    b.q[0], b.k[0], b.v[0] = a.q[0], a.k[0], a.v[0]
+    oa, ob = _run(a).cpu(), _run(b).cpu()
+    assert torch.equal(oa[0], ob[0])
+
+
+def test_deterministic_repeat():
+    case = syn.encoder_case(1, 4, 700, 64, seed=98)
+    assert torch.equal(_run(case).cpu(), _run(case).cpu())

@@ -1,0 +1,94 @@
+"""CPU-side checks of the C-ABI library: it builds, loads without a GPU, and
+exports every function include/attn.h declares; host-side validation."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from online_softmax_attention_flash_b200 import binding as B
+from online_softmax_attention_flash_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load_library()
+
+
+def test_header_declares_the_three_entry_points():
+    names = _declared_functions()
+    for n in ("attn_encoder_fwd", "attn_gqa_decode", "attn_paged_history", "attn_check",
+              "attn_gqa_decode_workspace_size"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in _declared_functions():
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_binding_signatures_cover_the_header():
+    assert sorted(n for n, _, _ in B.SIGNATURES) == _declared_functions()
+
+
+def test_nothing_else_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    ours = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert ours == set(_declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.attn_version() == 10000
+    assert lib.attn_status_string(-8) == b"ATTN_ERR_BLOCK_TABLE"
+    assert lib.attn_status_string(0) == b"ATTN_OK"
+
+
+def test_host_validation_rejects_before_any_launch(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)   # never dereferenced: validation fails first
+    # null pointers
+    assert lib.attn_encoder_fwd(None, fake, fake, fake, 1, 1, 128, 64, 0.125, None, None) == -1
+    # bad head_dim / shape / scale / alignment
+    assert lib.attn_encoder_fwd(fake, fake, fake, fake, 1, 1, 128, 96, 0.125, None, None) == -3
+    assert lib.attn_encoder_fwd(fake, fake, fake, fake, 0, 1, 128, 64, 0.125, None, None) == -2
+    assert lib.attn_encoder_fwd(fake, fake, fake, fake, 1, 1, 128, 64, -1.0, None, None) == -2
+    assert lib.attn_encoder_fwd(fake, fake, fake, P(4098), 1, 1, 128, 64, 0.1, None, None) == -4
+    # decode: group mismatch, head_dim, workspace
+    assert lib.attn_gqa_decode(fake, fake, fake, None, fake, 2, 16, 8, 3, 64, 256, 1.0, fake,
+                               1 << 20, None) == -2
+    assert lib.attn_gqa_decode(fake, fake, fake, None, fake, 2, 16, 8, 2, 64, 96, 1.0, fake,
+                               1 << 20, None) == -3
+    assert lib.attn_gqa_decode(fake, fake, fake, None, fake, 2, 16, 8, 2, 64, 256, 1.0, fake,
+                               16, None) == -5
+    # paged: block size, history length beyond the table, head_dim
+    args = dict(n_table=4, nb=4, bs=512, L=100, D=256)
+    def paged(bs=512, L=100, D=256, n_table=4):
+        return lib.attn_paged_history(fake, fake, fake, fake, n_table, 4, bs, L, 1.0, 1.0, 0.0625,
+                                      32, 2, 16, 64, D, fake, None)
+    assert paged(bs=500) == -2
+    assert paged(bs=640) == -2
+    assert paged(L=4 * 512 + 1) == -2
+    assert paged(D=192) == -3
+
+
+def test_workspace_size_query(lib):
+    n = lib.attn_gqa_decode_workspace_size(8, 16, 8, 4096, 256)
+    # 16 key splits of 256, fp32 o [B,Hq,16,D] + m, l
+    assert n >= 8 * 16 * 16 * 256 * 4 + 2 * 8 * 16 * 16 * 4
+    assert lib.attn_gqa_decode_workspace_size(8, 15, 8, 4096, 256) == 0
