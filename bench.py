@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the online-softmax attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Default workload ("vitl"): V-JEPA2 ViT-L encoder attention, B=1, H=16, S=2048,
+D=64, bf16, scale 1/8; one step = the 24 layers' worth of independent calls
+(24 distinct seeded input sets, 384 MiB per step, so every call's inputs come
+from HBM: the inputs are larger than the 126 MB L2). Other workloads:
+"tiny", "dinov3", "decode" (GQA decode, HBM bound, 4 rotating input sets),
+"paged" (history-only attention over the FP8 paged cache).
+
+Output: ONE JSON line on rank 0. `value` is whole-job throughput over all ranks
+(attention TFLOP/s, or GB/s for decode) with inputs resident in HBM, timed with
+CUDA events on the launching stream between barriers, max over ranks. `e2e` is
+the same metric through the public API with pinned host buffers (host->device
+copies of the step's inputs and device->host copies of its outputs inside the
+timed region). `roofline` relates the dominant kernel to the measured peak in
+MEASURED_PEAKS.json. `cpu_baseline` times the fp64 CPU oracle on a bounded
+sample (rank 0, N=1 only).
+
+Multi-GPU: launched by torchrun, one process per GPU; every rank runs the same
+workload on its own GPU (independent problems, no data-path collective), so
+scaling is weak.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s (encoder/prefill) & KV GB/s (decode) vs B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    "vitl": dict(kind="encoder", B=1, H=16, S=2048, D=64, scale=0.125, sets=24, seed0=2000,
+                 name="vitl_b1_h16_s2048_d64_x24layers"),
+    "tiny": dict(kind="encoder", B=1, H=4, S=256, D=64, scale=0.125, sets=1, seed0=1001,
+                 name="tiny_mha_b1_h4_s256_d64"),
+    "dinov3": dict(kind="encoder", B=8, H=16, S=201, D=64, scale=0.125, sets=1, seed0=1003,
+                   name="dinov3_b8_h16_s201_d64"),
+    "decode": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=256, scale=1.0, sets=4,
+                   seed0=1004, name="gqa_decode_b8_16q_8kv_d256_ctx4096"),
+    "paged": dict(kind="paged", Hq=32, Hkv=2, Sq=4096, D=256, NB=256, BS=512, L=100000,
+                  scale=1.0 / 16, sets=1, seed0=1005,
+                  name="paged_history_32q_2kv_d256_q4096_hist100000_fp8"),
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic(kernel_regex: str, workload: str):
+    """DRAM bytes per launch from profiles/dram_traffic.txt, if captured on this build."""
+    from online_softmax_attention_flash_b200.build import source_digest
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#"):
+                if parts[0] == kernel_regex and parts[1] == workload and parts[3] == digest:
+                    return int(parts[2])
+    return None
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_smi_id(device) -> str:
+    """nvidia-smi -i accepts a GPU UUID; CUDA_VISIBLE_DEVICES may renumber indices."""
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        return str(device.index or 0)
+
+
+# ------------------------------------------------------------------ workloads
+class EncoderWork:
+    def __init__(self, cfg, device):
+        import torch
+        from online_softmax_attention_flash_b200 import inputs as syn
+        self.cfg = cfg
+        self.sets = []
+        self.host = []
+        for i in range(cfg["sets"]):
+            c = syn.encoder_case(cfg["B"], cfg["H"], cfg["S"], cfg["D"], seed=cfg["seed0"] + i,
+                                 softmax_scale=cfg["scale"])
+            self.host.append(c)
+            self.sets.append(tuple(t.to(device) for t in (c.q, c.k, c.v)))
+        self.out = [torch.empty_like(s[0]) for s in self.sets]
+        B, H, S, D = cfg["B"], cfg["H"], cfg["S"], cfg["D"]
+        self.flops_per_launch = 4.0 * B * H * S * S * D
+        self.launches_per_step = cfg["sets"]
+        self.work_per_step = self.flops_per_launch * cfg["sets"]
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.kernel_regex = "encoder_fwd_kernel"
+
+    def step(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        for (q, k, v), o in zip(self.sets, self.out):
+            Bd.attn_encoder_fwd(q, k, v, self.cfg["scale"], out=o, stream=stream)
+
+    def rate(self, work, seconds):
+        return work / seconds / 1e12
+
+    # end-to-end through the public API with pinned host buffers
+    def e2e_setup(self):
+        import torch
+        self.h_in = [tuple(t.pin_memory() for t in (c.q, c.k, c.v)) for c in self.host]
+        self.h_out = [torch.empty_like(c.q).pin_memory() for c in self.host]
+        self.h2d = sum(t.numel() * t.element_size() for s in self.h_in for t in s)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        for (hq, hk, hv), (q, k, v), o, ho in zip(self.h_in, self.sets, self.out, self.h_out):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            Bd.attn_encoder_fwd(q, k, v, self.cfg["scale"], out=o, stream=stream)
+            ho.copy_(o, non_blocking=True)
+
+    # CPU oracle on a bounded sample of the same workload
+    def oracle_sample(self, step_idx, rows=256):
+        import oracle
+        c = self.host[step_idx % len(self.host)]
+        S = self.cfg["S"]
+        h = step_idx % self.cfg["H"]
+        r0 = (step_idx * rows) % max(1, S - rows + 1) if S > rows else 0
+        rr = np.arange(r0, min(S, r0 + rows))
+        q = c.q[0:1, h:h + 1].double().numpy()
+        k = c.k[0:1, h:h + 1].double().numpy()
+        v = c.v[0:1, h:h + 1].double().numpy()
+        oracle.encoder_attention(q, k, v, self.cfg["scale"], rows=rr)
+        return 4.0 * len(rr) * S * self.cfg["D"], f"{len(rr)} query rows x {S} keys of one head"
+
+
+class DecodeWork:
+    def __init__(self, cfg, device):
+        import torch
+        from online_softmax_attention_flash_b200 import binding as Bd
+        from online_softmax_attention_flash_b200 import inputs as syn
+        import oracle
+        self.cfg = cfg
+        self.host, self.sets = [], []
+        for i in range(cfg["sets"]):
+            c = syn.decode_case(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"],
+                                seed=cfg["seed0"] + 100 * i, softmax_scale=cfg["scale"])
+            self.host.append(c)
+            self.sets.append(tuple(t.to(device) for t in (c.q, c.k, c.v, c.attn_mask)))
+        self.out = [torch.empty_like(s[0]) for s in self.sets]
+        ws = Bd.attn_gqa_decode_workspace_size(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"])
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.bytes = [oracle.decode_algorithmic_bytes(c.lengths.tolist(), cfg["Hkv"], cfg["D"],
+                                                      cfg["Hq"], cfg["S"]) for c in self.host]
+        self.launches_per_step = 2   # split + combine
+        self.work_per_step = float(np.mean(self.bytes))
+        self.flops_per_launch = self.work_per_step
+        self.unit, self.bound = "GB/s", "hbm"
+        self.kernel_regex = "decode_split_kernel"
+        self.i = 0
+
+    def step(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        j = self.i % len(self.sets)
+        self.i += 1
+        q, k, v, m = self.sets[j]
+        Bd.attn_gqa_decode(q, k, v, m, self.cfg["scale"], self.cfg["Hq"] // self.cfg["Hkv"],
+                           out=self.out[j], workspace=self.ws, stream=stream)
+
+    def rate(self, work, seconds):
+        return work / seconds / 1e9
+
+    def e2e_setup(self):
+        import torch
+        c = self.host[0]
+        self.h_in = tuple(t.pin_memory() for t in (c.q, c.k, c.v, c.attn_mask))
+        self.h_out = torch.empty_like(c.q).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def e2e_step(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        q, k, v, m = self.sets[0]
+        for d, h in zip((q, k, v, m), self.h_in):
+            d.copy_(h, non_blocking=True)
+        Bd.attn_gqa_decode(q, k, v, m, self.cfg["scale"], self.cfg["Hq"] // self.cfg["Hkv"],
+                           out=self.out[0], workspace=self.ws, stream=stream)
+        self.h_out.copy_(self.out[0], non_blocking=True)
+
+    def e2e_work(self):
+        return self.bytes[0]
+
+    def oracle_sample(self, step_idx):
+        import oracle
+        c = self.host[step_idx % len(self.host)]
+        b = step_idx % self.cfg["B"]
+        oracle.gqa_decode_attention(c.q[b:b + 1].double().numpy(), c.k[b:b + 1].double().numpy(),
+                                    c.v[b:b + 1].double().numpy(),
+                                    c.attn_mask[b:b + 1].double().numpy(), self.cfg["scale"],
+                                    self.cfg["Hq"] // self.cfg["Hkv"])
+        L = int(c.lengths[b])
+        byt = L * self.cfg["Hkv"] * self.cfg["D"] * 4 + 2 * self.cfg["Hq"] * self.cfg["D"] * 2
+        return float(byt), "one batch entry (all heads) of the decode step"
+
+
+class PagedWork:
+    def __init__(self, cfg, device):
+        import torch
+        from online_softmax_attention_flash_b200 import inputs as syn
+        self.cfg = cfg
+        c = syn.paged_case(cfg["Hq"], cfg["Hkv"], cfg["Sq"], cfg["D"], cfg["NB"], cfg["BS"],
+                           cfg["L"], seed=cfg["seed0"], softmax_scale=cfg["scale"])
+        self.host = [c]
+        self.dev = tuple(t.to(device) for t in (c.q, c.k_cache, c.v_cache, c.block_table))
+        self.out = torch.empty_like(self.dev[0])
+        self.flops_per_launch = 4.0 * cfg["Sq"] * cfg["Hq"] * cfg["L"] * cfg["D"]
+        self.launches_per_step = 1
+        self.work_per_step = self.flops_per_launch
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.kernel_regex = "paged_history_kernel"
+
+    def _call(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        c = self.host[0]
+        q, kc, vc, bt = self.dev
+        Bd.attn_paged_history(q, kc, vc, bt, c.block_size, c.actual_history_len, c.k_scale,
+                              c.v_scale, c.softmax_scale, c.num_kv_groups, out=self.out,
+                              stream=stream)
+
+    def step(self, stream):
+        self._call(stream)
+
+    def rate(self, work, seconds):
+        return work / seconds / 1e12
+
+    def e2e_setup(self):
+        import torch
+        c = self.host[0]
+        self.h_in = tuple(t.pin_memory() for t in (c.q, c.k_cache, c.v_cache, c.block_table))
+        self.h_out = torch.empty_like(c.q).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def e2e_step(self, stream):
+        for d, h in zip(self.dev, self.h_in):
+            d.copy_(h, non_blocking=True)
+        self._call(stream)
+        self.h_out.copy_(self.out, non_blocking=True)
+
+    def oracle_sample(self, step_idx, rows=16):
+        import oracle
+        c = self.host[0]
+        h = step_idx % self.cfg["Hq"]
+        r0 = (step_idx * rows) % self.cfg["Sq"]
+        rr = np.arange(r0, min(self.cfg["Sq"], r0 + rows))
+        # one query head against its kv head only
+        g = h // c.num_kv_groups
+        oracle.paged_history_attention(c.q[h:h + 1].double().numpy(),
+                                       c.k_cache[:, g:g + 1].numpy(), c.v_cache[:, g:g + 1].numpy(),
+                                       c.k_scale, c.v_scale, c.block_table.numpy(), c.block_size,
+                                       c.actual_history_len, c.softmax_scale, 1, rows=rr)
+        return 4.0 * len(rr) * self.cfg["L"] * self.cfg["D"], f"{len(rr)} query rows of one head"
+
+
+def make_work(name, device):
+    cfg = WORKLOADS[name]
+    return {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork}[cfg["kind"]](cfg, device)
+
+
+# --------------------------------------------------------------------- oracle
+def cpu_oracle_run(work, budget_s: float, max_steps=None, start=0):
+    """Time the oracle (as it stands) on a bounded sample; returns (rate, secs, sample, steps)."""
+    done, total, n, sample = 0.0, 0.0, 0, ""
+    t_end = time.perf_counter() + budget_s
+    while True:
+        t0 = time.perf_counter()
+        w, sample = work.oracle_sample(start + n)
+        total += time.perf_counter() - t0
+        done += w
+        n += 1
+        if (max_steps is not None and n >= max_steps) or (max_steps is None and time.perf_counter() > t_end):
+            break
+    return work.rate(done, total), total, sample, n
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- arms
+def run_reference(args, info):
+    """The reference arm: the fp64 CPU oracle timed on the host cores (rank 0 only)."""
+    if not info.is_main:
+        return 0
+    cfg = WORKLOADS[args.workload]
+    work = make_work_host_only(args.workload)
+    for i in range(args.warmup):
+        work.oracle_sample(i)
+    rate, secs, sample, n = cpu_oracle_run(work, 0, max_steps=args.steps, start=args.warmup)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": work.unit,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(1, n), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg["name"], "sample_per_step": sample},
+        "cpu_baseline": {"value": rate, "unit": work.unit, "cores": cores(), "kind": "oracle",
+                         "sample": f"each step: {sample}"},
+        "e2e": {"value": rate, "unit": work.unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def make_work_host_only(name):
+    """Host-side inputs only (the oracle arm never touches a GPU)."""
+    cfg = WORKLOADS[name]
+    cls = {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork}[cfg["kind"]]
+    obj = cls.__new__(cls)
+    obj.cfg = cfg
+    from online_softmax_attention_flash_b200 import inputs as syn
+    if cfg["kind"] == "encoder":
+        obj.host = [syn.encoder_case(cfg["B"], cfg["H"], cfg["S"], cfg["D"], seed=cfg["seed0"] + i,
+                                     softmax_scale=cfg["scale"]) for i in range(cfg["sets"])]
+        obj.unit = "TFLOP/s"
+    elif cfg["kind"] == "decode":
+        obj.host = [syn.decode_case(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"],
+                                    seed=cfg["seed0"] + 100 * i, softmax_scale=cfg["scale"])
+                    for i in range(cfg["sets"])]
+        obj.unit = "GB/s"
+    else:
+        obj.host = [syn.paged_case(cfg["Hq"], cfg["Hkv"], cfg["Sq"], cfg["D"], cfg["NB"], cfg["BS"],
+                                   cfg["L"], seed=cfg["seed0"], softmax_scale=cfg["scale"])]
+        obj.unit = "TFLOP/s"
+    return obj
+
+
+def run_product(args, info):
+    import torch
+    from online_softmax_attention_flash_b200 import binding as Bd
+    from online_softmax_attention_flash_b200 import dist as D
+
+    torch.cuda.set_device(info.local_rank)
+    device = torch.device("cuda", info.local_rank)
+    Bd.load_library()
+    work = make_work(args.workload, device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(args.warmup):
+        work.step(stream)
+    torch.cuda.synchronize(device)
+    st = Bd.attn_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {Bd.STATUS.get(st, st)}")
+
+    sampler = ClockSampler(gpu_smi_id(device))
+    sampler.start()
+    time.sleep(0.2)
+    D.barrier(info)
+    torch.cuda.synchronize(device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        work.step(stream)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    D.barrier(info)
+    clocks = sampler.stop()
+    step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    st = Bd.attn_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {Bd.STATUS.get(st, st)}")
+    max_ms = D.max_over_ranks(total_ms, info, device)
+
+    work_all = work.work_per_step * args.steps * info.world_size
+    value = work.rate(work_all, max_ms / 1e3)
+
+    # roofline of the dominant kernel: algorithmic work per launch / mean launch time
+    peaks, peak_src = load_peaks()
+    per_launch_ms = total_ms / (args.steps * work.launches_per_step)
+    if work.bound == "hbm":
+        # decode: one call = split + combine; achieved counts the whole call's time
+        per_call_ms = total_ms / args.steps
+        achieved = work.work_per_step / (per_call_ms / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        peak_name = "hbm_gbs"
+    else:
+        achieved = work.flops_per_launch / (per_launch_ms / 1e3) / 1e12
+        sustained = total_ms > 1000.0
+        peak_name = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+        peak = float(peaks[peak_name])
+    roofline = {"bound": work.bound, "achieved": achieved, "peak": peak, "unit": work.unit,
+                "frac": achieved / peak,
+                "traffic": profiled_traffic(work.kernel_regex, args.workload),
+                "peak_source": f"{peak_src} ({peak_name})", "kernel": work.kernel_regex}
+
+    # end to end through the public API with host buffers
+    work.e2e_setup()
+    e2e_steps = max(1, min(args.steps, 10))
+    work.e2e_step(stream)
+    torch.cuda.synchronize(device)
+    D.barrier(info)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        work.e2e_step(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), info, device)
+    e2e_work = getattr(work, "e2e_work", lambda: work.work_per_step)()
+    e2e = {"value": work.rate(e2e_work * e2e_steps * info.world_size, e2e_ms / 1e3),
+           "unit": work.unit, "h2d_bytes_per_step": int(work.h2d),
+           "d2h_bytes_per_step": int(work.d2h), "steps": e2e_steps}
+
+    if not info.is_main:
+        return 0
+    cpu = None
+    if info.world_size == 1 and not args.no_cpu_baseline:
+        rate, secs, sample, n = cpu_oracle_run(work, args.cpu_budget)
+        cpu = {"value": rate, "unit": work.unit, "cores": cores(), "kind": "oracle",
+               "sample": f"{n} samples of {sample} ({secs:.1f} s of fp64 NumPy)"}
+    cfg = WORKLOADS[args.workload]
+    s_sorted = sorted(step_ms)
+    line = {
+        "metric": METRIC, "value": value, "unit": work.unit, "n_gpus": info.world_size,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg["name"],
+                   **{k: v for k, v in cfg.items() if k not in ("kind", "name", "seed0")},
+                   "l2": ("inputs larger than L2: distinct input sets rotate across calls"
+                          if cfg["sets"] > 1 or cfg["kind"] == "paged" else "inputs fit in L2"),
+                   "parallelism": f"replicas x{info.world_size}"},
+        "step_ms": {"min": s_sorted[0], "median": statistics.median(step_ms),
+                    "mean": statistics.fmean(step_ms),
+                    "p90": s_sorted[min(len(s_sorted) - 1, int(0.9 * len(s_sorted)))],
+                    "max": s_sorted[-1]},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * work.launches_per_step,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=None)
+    p.add_argument("--workload", default="vitl", choices=sorted(WORKLOADS))
+    p.add_argument("--impl", default="product", choices=["product", "reference"])
+    p.add_argument("--cpu-budget", type=float, default=12.0,
+                   help="seconds of oracle work for cpu_baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    defaults = {"vitl": (1000, 20), "tiny": (2000, 20), "dinov3": (2000, 20),
+                "decode": (2000, 20), "paged": (100, 5)}[args.workload]
+    if args.steps is None:
+        args.steps = defaults[0]
+    if args.warmup is None:
+        args.warmup = defaults[1]
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    from online_softmax_attention_flash_b200 import dist as D
+    info = D.rank_info_from_env()
+    if args.impl == "reference":
+        # the oracle arm runs on rank 0 only; other ranks exit without work
+        return run_reference(args, info)
+    info = D.init("nccl" if info.world_size > 1 else "gloo")
+    if info.world_size != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={info.world_size}")
+    try:
+        return run_product(args, info)
+    finally:
+        D.shutdown(info)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -34,6 +34,17 @@ def sources():
                   if f.endswith((".cu", ".cuh")))
 
 
+def source_digest() -> str:
+    """sha256 over the library's CUDA sources and header (identifies a kernel build)."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in sources() + [os.path.join(INCLUDE, "attn.h")]:
+        h.update(os.path.basename(path).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def up_to_date() -> bool:
     if not os.path.exists(LIB_PATH):
         return False
