@@ -115,6 +115,42 @@ ATTN_API int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_
                     void* stream);
 
 /*
+ * attn_gqa_decode_noalloc -- attn_gqa_decode for callers that cannot allocate
+ * device memory.
+ *
+ * The pages have no counterpart of this function; it exists for deployment.
+ * Some hosts own the whole device-memory budget and forbid allocations after
+ * start-up (plugin and embedded runtimes), and some latency-critical loops
+ * cannot afford cudaMalloc, which may synchronise the whole device. Such
+ * callers cannot provide the workspace attn_gqa_decode needs. This entry point
+ * computes exactly what attn_gqa_decode computes (same kernels, same results)
+ * but keeps the split-KV partials in a scratch array that the library reserves
+ * statically on every device that loads it (ATTN_NOALLOC_SCRATCH_BYTES, held
+ * until the process exits). It calls no allocator.
+ *
+ *   Arguments: as attn_gqa_decode, without the workspace pair. The caller
+ *   still owns q, k, v, attn_mask and out.
+ *   Limit: attn_gqa_decode_workspace_size(B, Hq, Hkv, S_ctx, D) must not
+ *   exceed ATTN_NOALLOC_SCRATCH_BYTES; larger problems are rejected with
+ *   ATTN_ERR_WORKSPACE before anything is enqueued.
+ *   Set-up: the first call on a device looks up the scratch array's device
+ *   address on the current device (once per device). Make that first call
+ *   outside any stream capture.
+ *   Sharing: all calls on a device use the same scratch array, which keeps the
+ *   previous call's contents (nothing in it needs to start at zero). Calls that
+ *   may run at the same time on the GPU (different streams without ordering)
+ *   race on it: order them on one stream, or use attn_gqa_decode with separate
+ *   workspaces.
+ * Errors: as attn_gqa_decode; ATTN_ERR_WORKSPACE when the sizes exceed the
+ * scratch; ATTN_ERR_CUDA if the address look-up fails.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+ATTN_API int attn_gqa_decode_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     const float* attn_mask, uint16_t* out,
+                                     int B, int Hq, int Hkv, int num_kv_groups, int S_ctx, int D,
+                                     float softmax_scale, void* stream);
+
+/*
  * attn_paged_history -- history-only attention over a paged FP8 KV cache.
  *
  * Defined by: "Prefill Context-Parallel Attention POC for Trainium2",

@@ -35,6 +35,7 @@ SIGNATURES = [
     ("attn_encoder_fwd", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
     ("attn_gqa_decode_workspace_size", _SZ, [_I, _I, _I, _I, _I]),
     ("attn_gqa_decode", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _SZ, _P]),
+    ("attn_gqa_decode_noalloc", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     ("attn_paged_history", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _I, _I, _I, _I, _I,
                                 _P, _P]),
     ("attn_check", _I, [_P]),
@@ -153,6 +154,36 @@ def attn_gqa_decode(q, k, v, attn_mask, softmax_scale: float, num_kv_groups: int
                              int(num_kv_groups), S_ctx, D, float(softmax_scale), _ptr(workspace),
                              workspace.numel(), _stream_ptr(stream))
     _raise_if(st, "attn_gqa_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024   # ATTN_NOALLOC_SCRATCH_BYTES in include/attn.h
+
+
+def attn_gqa_decode_noalloc(q, k, v, attn_mask, softmax_scale: float, num_kv_groups: int,
+                            out=None, stream=None):
+    """attn_gqa_decode without a caller workspace: the partials live in the
+    library's static per-device scratch (for callers that cannot allocate).
+    Calls that may overlap on the GPU share that scratch and race."""
+    lib = load_library()
+    _need(q, "q", torch.bfloat16)
+    B, Hq, one, D = q.shape
+    if one != 1:
+        raise ValueError("q must be [B, Hq, 1, D] (single-token decode)")
+    _need(k, "k", torch.bfloat16)
+    Bk, Hkv, S_ctx, Dk = k.shape
+    if Bk != B or Dk != D:
+        raise ValueError("k must be [B, Hkv, S_ctx, D]")
+    _need(v, "v", torch.bfloat16, k.shape)
+    if attn_mask is not None:
+        _need(attn_mask, "attn_mask", torch.float32, (B, 1, 1, S_ctx))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, q.shape)
+    st = lib.attn_gqa_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(attn_mask), _ptr(out), B,
+                                     Hq, Hkv, int(num_kv_groups), S_ctx, D, float(softmax_scale),
+                                     _stream_ptr(stream))
+    _raise_if(st, "attn_gqa_decode_noalloc")
     return out
 
 

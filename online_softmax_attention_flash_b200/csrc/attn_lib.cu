@@ -98,6 +98,29 @@ int launch_encoder(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Scratch for attn_gqa_decode_noalloc: reserved statically on every device that
+// loads this library, so that entry point never allocates. Host code must not
+// use the symbol as an address; it looks up the device address once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -172,6 +195,20 @@ int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
     return attn::dec::launch(q, k, v, attn_mask, out, B, Hq, Hkv, num_kv_groups, S_ctx, D,
                              softmax_scale, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int attn_gqa_decode_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            const float* attn_mask, uint16_t* out, int B, int Hq, int Hkv,
+                            int num_kv_groups, int S_ctx, int D, float softmax_scale,
+                            void* stream) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || S_ctx < 1 || Hq % Hkv) return ATTN_ERR_SHAPE;
+    const size_t need = attn::dec::workspace_bytes(B, Hq, S_ctx, D);
+    if (need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    return attn_gqa_decode(q, k, v, attn_mask, out, B, Hq, Hkv, num_kv_groups, S_ctx, D,
+                           softmax_scale, scratch, ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,

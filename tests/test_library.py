@@ -92,3 +92,11 @@ def test_workspace_size_query(lib):
     # 16 key splits of 256, fp32 o [B,Hq,16,D] + m, l
     assert n >= 8 * 16 * 16 * 256 * 4 + 2 * 8 * 16 * 16 * 4
     assert lib.attn_gqa_decode_workspace_size(8, 15, 8, 4096, 256) == 0
+
+
+def test_noalloc_size_limit_is_checked_on_the_host(lib):
+    fake = ctypes.c_void_p(4096)
+    assert lib.attn_gqa_decode_noalloc(fake, fake, fake, None, fake, 64, 64, 8, 8, 65536, 512,
+                                       1.0, None) == -5
+    assert lib.attn_gqa_decode_noalloc(fake, fake, fake, None, fake, 0, 16, 8, 2, 64, 256,
+                                       1.0, None) == -2

@@ -1,0 +1,57 @@
+"""The allocation-free decode entry point, attn_gqa_decode_noalloc.
+
+Some callers cannot allocate device memory: hosts that own the whole memory
+budget and forbid allocations once they are running, and latency-critical
+loops that cannot pay for cudaMalloc's possible device-wide synchronisation.
+They cannot hand attn_gqa_decode a workspace, so the library offers a variant
+whose split-KV partials live in a scratch array reserved statically on the
+device. These tests call it through the C ABI and check that it returns what
+the workspace-taking entry point returns, twice in a row (the scratch keeps the
+previous call's contents, so the second call must not be affected by the first).
+
+This file is named so that pytest collects it last.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+from online_softmax_attention_flash_b200 import binding as B
+from online_softmax_attention_flash_b200 import inputs as syn
+from parity import BF16_HEAD_COS, BF16_REL_L2, head_cosines, rel_l2, to_f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _device_case(case):
+    return tuple(t.to(DEV) for t in (case.q, case.k, case.v, case.attn_mask))
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    cases = [syn.decode_case(8, 16, 8, 4096, 256, seed=4242, softmax_scale=1.0),
+             syn.decode_case(3, 8, 2, 1500, 512, seed=4343, softmax_scale=512 ** -0.5,
+                             min_len=1)]
+    for case in cases:   # two calls in a row, different sizes and contents
+        q, k, v, m = _device_case(case)
+        need = B.attn_gqa_decode_workspace_size(q.shape[0], q.shape[1], k.shape[1], k.shape[2],
+                                                q.shape[3])
+        assert need <= B.NOALLOC_SCRATCH_BYTES
+        ref = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups)
+        got = B.attn_gqa_decode_noalloc(q, k, v, m, case.softmax_scale, case.num_kv_groups)
+        assert B.attn_check() == 0
+        g, r = to_f64(got), to_f64(ref)
+        assert rel_l2(g, r) <= BF16_REL_L2
+        assert head_cosines(g, r, 2).min() >= BF16_HEAD_COS
+
+
+def test_noalloc_rejects_sizes_beyond_the_scratch():
+    lib = B.load_library()
+    fake = ctypes.c_void_p(4096)   # never dereferenced: the size check comes first
+    # 64 x 64 heads x 256 splits x 512 floats is far beyond the 4 MiB scratch
+    st = lib.attn_gqa_decode_noalloc(fake, fake, fake, None, fake, 64, 64, 8, 8, 65536, 512,
+                                     1.0, None)
+    assert st == -5   # ATTN_ERR_WORKSPACE
+    torch.cuda.synchronize()
