@@ -170,7 +170,8 @@ ATTN_API int attn_gqa_decode_noalloc(const uint16_t* q, const uint16_t* k, const
  *   actual_history_len : 0 <= len <= n_table * block_size. Positions >= len
  *                  are ignored (a partial last block is allowed); blocks
  *                  wholly beyond len are never read.
- *   k_scale, v_scale   : per-tensor dequantisation scales (value = code * scale)
+ *   k_scale, v_scale   : per-tensor dequantisation scales (value = code * scale);
+ *                  k_scale finite and > 0, v_scale finite
  *   out          : [Hq, Sq, D] bf16
  *   Hq == Hkv * num_kv_groups; D == 256; block_size in {128, 256, 384, 512}.
  *   Every query attends to every history position < len (no causal mask).

@@ -18,43 +18,11 @@
 #include "decode.cuh"
 #include "encoder.cuh"
 #include "paged.cuh"
+#include "tmap.cuh"
 
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
-
-// ------------------------------------------------------------ driver entry
-PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
-std::once_flag g_encode_once;
-
-bool load_encode_tiled() {
-    std::call_once(g_encode_once, [] {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    return g_encode_tiled != nullptr;
-}
-
-// Tiled map over a rank-3 row-major tensor [d2][d1][d0] with a 128-byte swizzle.
-// elem_bytes * box0 must be 128 (one swizzle row).
-int encode_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t elem_bytes,
-                  const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
-                  uint32_t box1) {
-    if (!load_encode_tiled()) return ATTN_ERR_CUDA;
-    cuuint64_t dims[3] = {d0, d1, d2};
-    cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
-    cuuint32_t box[3] = {box0, box1, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode_tiled(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
-}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -85,12 +53,9 @@ int launch_encoder(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint
     CUtensorMap tq, tk, tv;
     const uint64_t rows = static_cast<uint64_t>(S);
     const uint64_t heads = static_cast<uint64_t>(B) * H;
-    if ((rc = encode_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, D, rows, heads, 64, kTileM)))
-        return rc;
-    if ((rc = encode_map_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, D, rows, heads, 64, kTileN)))
-        return rc;
-    if ((rc = encode_map_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, D, rows, heads, 64, kTileN)))
-        return rc;
+    if ((rc = attn::encode_map_3d_bf16(&tq, q, D, rows, heads, 64, kTileM))) return rc;
+    if ((rc = attn::encode_map_3d_bf16(&tk, k, D, rows, heads, 64, kTileN))) return rc;
+    if ((rc = attn::encode_map_3d_bf16(&tv, v, D, rows, heads, 64, kTileN))) return rc;
     dim3 grid((S + kRowsPerCta - 1) / kRowsPerCta, static_cast<unsigned>(heads));
     const float scale_log2 = scale * kLog2e;
     kernel<<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, out, key_bias, H, S,
@@ -223,7 +188,7 @@ int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const uint8_t*
     if (block_size < 128 || block_size > 512 || block_size % 128) return ATTN_ERR_SHAPE;
     if (static_cast<int64_t>(actual_history_len) > static_cast<int64_t>(n_table) * block_size)
         return ATTN_ERR_SHAPE;
-    if (!scale_ok(softmax_scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    if (!scale_ok(softmax_scale) || !scale_ok(k_scale) || !std::isfinite(v_scale))
         return ATTN_ERR_SHAPE;
     if (D != 256) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||

@@ -1,0 +1,56 @@
+// tmap.cuh -- host-side TMA tensor-map encoding (driver entry point fetched through
+// the runtime, so the library does not link libcuda directly).
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+namespace attn {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tiled map over a rank-3 row-major tensor [d2][d1][d0] with the 128-byte swizzle
+// (box0 * elem_bytes must be 128). Out-of-range box elements read as zero.
+// Returns 0 or -6 (ATTN_ERR_CUDA).
+inline int encode_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t elem_bytes,
+                         const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                         uint32_t box1) {
+    auto fn = encode_tiled_fn();
+    if (!fn) return -6;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -6;
+}
+
+inline int encode_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint32_t box0, uint32_t box1) {
+    return encode_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d0, d1, d2, box0, box1);
+}
+
+inline int encode_map_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                            uint64_t d2, uint32_t box0, uint32_t box1) {
+    return encode_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, d0, d1, d2, box0, box1);
+}
+
+}  // namespace attn
