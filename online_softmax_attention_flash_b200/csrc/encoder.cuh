@@ -31,9 +31,19 @@ constexpr int kTileM = 128;            // query rows per tile = TMEM lanes
 constexpr int kTileN = 128;            // keys per K/V tile
 constexpr int kQTiles = 2;             // query tiles per CTA
 constexpr int kRowsPerCta = kTileM * kQTiles;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;          // 8 softmax warps + producer + MMA
+// Warps 0-15 run the softmax: warp w serves query tile w / 8, half (w / 4) % 2 of the
+// 128 S columns, TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31. Two warps share every row, so
+// each scheduler holds four softmax warps to hide TMEM / MUFU / barrier latency.
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 576;
+#ifndef ATTN_ENC_POLY_EIGHTHS
+#define ATTN_ENC_POLY_EIGHTHS 3
+#endif
+// Of every 8 column pairs of an unmasked S tile, this many take 2^x from the FMA-pipe
+// polynomial instead of the MUFU ex2 unit (which alone caps D=64 at half the MMA rate).
+constexpr int kPolyEighths = ATTN_ENC_POLY_EIGHTHS;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -48,13 +58,21 @@ struct Cfg {
     static constexpr int kKOff = kQOff + kQTiles * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_final
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
+    // o_final, xchg[2] (row-max / row-sum exchange between the two halves of a tile),
+    // s_free[2] (softmax has read S_t), pv_done[2] (PV_t has completed)
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 2 + 2;
+    static constexpr int kXchgOff = kBarOff + kNumBars * 8;   // float [2 buf][2 tile][2 half][128]
+    static constexpr int kMiscOff = kXchgOff + 2 * 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + tmem slot, abort flag, alignment slack
-    // TMEM columns
+    // TMEM columns: S_t at 128 t, O_t at 256 + D t. For D = 64 the P tiles (bf16 pairs,
+    // 64 columns each) get their own columns at 384 + 64 t, so the next QK can overwrite
+    // S_t as soon as the softmax has read it; for D = 128 TMEM is full and P_t is written
+    // over the first 64 columns of S_t.
     static constexpr uint32_t kColS0 = 0;
     static constexpr uint32_t kColO0 = 256;
+    static constexpr bool kSepP = (D == 64);
+    static constexpr uint32_t kColP0 = kSepP ? 256 + 2 * D : 0;
 };
 
 struct Bars {
@@ -66,6 +84,9 @@ struct Bars {
     uint64_t* s_full;
     uint64_t* p_ready;
     uint64_t* o_final;
+    uint64_t* xchg;
+    uint64_t* s_free;
+    uint64_t* pv_done;
 };
 
 template <int D>
@@ -81,6 +102,9 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
     r.s_full = r.v_empty + C::kStages;
     r.p_ready = r.s_full + 2;
     r.o_final = r.p_ready + 2;
+    r.xchg = r.o_final + 1;
+    r.s_free = r.xchg + 2;
+    r.pv_done = r.s_free + 2;
     return r;
 }
 
@@ -111,7 +135,10 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars.s_full[t], 1);
-            mbar_init(&bars.p_ready[t], kTileM);
+            mbar_init(&bars.p_ready[t], kSoftmaxWarps / 2);   // one arrival per softmax warp of the tile
+            mbar_init(&bars.xchg[t], kSoftmaxWarps / 2);
+            mbar_init(&bars.s_free[t], kSoftmaxWarps / 2);
+            mbar_init(&bars.pv_done[t], 1);
         }
         mbar_init(bars.o_final, 1);
         *abort_flag = 0;
@@ -179,26 +206,31 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const uint32_t v_addr = smem_u32(smem + C::kVOff);
             bool ok = mbar_wait(bars.q_full, 0, abort_flag);
 
+            // Descriptors are built once; a K-step or a ring stage only moves the start
+            // address, i.e. adds (bytes >> 4) to the low word.
+            const uint64_t dq = smem_desc(q_addr, 16, 1024);
+            const uint64_t dk = smem_desc(k_addr, 16, 1024);
+            const uint64_t dv = smem_desc(v_addr, C::kPanelBytes, 1024);
             // S_t = Q_t K_j^T : K-steps of 16 along D (32 bytes inside a 128-byte panel row)
             auto issue_qk = [&](int t, int st) {
-                const uint32_t qa = q_addr + t * C::kTileBytes;
-                const uint32_t ka = k_addr + st * C::kTileBytes;
+                const uint64_t qa = dq + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
+                const uint64_t ka = dk + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
+                const uint32_t d = tmem_base + C::kColS0 + t * 128;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
-                    mma_f16_ss(tmem_base + C::kColS0 + t * 128, smem_desc(qa + off, 16, 1024),
-                               smem_desc(ka + off, 16, 1024), idesc_qk, kk > 0);
+                    const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kPanelBytes + (kk % 4) * 32) >> 4);
+                    mma_f16_ss(d, qa + off, ka + off, idesc_qk, kk > 0);
                 }
             };
             // O_t += P_t V_j : A = P_t in TMEM (bf16 pairs over S_t columns), B = V (MN-major)
             auto issue_pv = [&](int t, int st, bool acc) {
-                const uint32_t va = v_addr + st * C::kTileBytes;
+                const uint64_t va = dv + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
+                const uint32_t d = tmem_base + C::kColO0 + t * D;
+                const uint32_t a = C::kSepP ? tmem_base + C::kColP0 + t * 64 : tmem_base + C::kColS0 + t * 128;
 #pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk) {
-                    mma_f16_ts(tmem_base + C::kColO0 + t * D, tmem_base + C::kColS0 + t * 128 + kk * 8,
-                               smem_desc(va + kk * 16 * 128, C::kPanelBytes, 1024), idesc_pv,
+                for (int kk = 0; kk < kTileN / 16; ++kk)
+                    mma_f16_ts(d, a + kk * 8, va + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                                (acc || kk > 0) ? 1u : 0u);
-                }
             };
 
             if (ok) ok = mbar_wait(&bars.k_full[0], 0, abort_flag);
@@ -210,6 +242,59 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tc_commit(&bars.s_full[1]);
                 tc_commit(&bars.k_empty[0]);
             }
+            if constexpr (C::kSepP) {
+                // Issue whichever MMA is ready: QK_t(j) needs K_j and the softmax to have read
+                // S_t(j-1); PV_t(j) needs V_j and P_t(j). The two query tiles progress
+                // independently; a K / V stage is released once both tiles have used it.
+                int qk_next[kQTiles] = {1, 1}, pv_next[kQTiles] = {0, 0};
+                int k_rel = 1, v_rel = 0;
+                uint64_t t_idle = 0;
+                uint32_t spins = 0;
+                while (ok && (pv_next[0] < n_kv || pv_next[1] < n_kv)) {
+                    bool progress = false;
+#pragma unroll
+                    for (int t = 0; t < kQTiles; ++t) {
+                        const int jq = qk_next[t];
+                        if (jq < n_kv && mbar_try_wait(&bars.s_free[t], (jq - 1) & 1) &&
+                            mbar_try_wait(&bars.k_full[jq % C::kStages], (jq / C::kStages) & 1)) {
+                            tc_fence_after();
+                            issue_qk(t, jq % C::kStages);
+                            tc_commit(&bars.s_full[t]);
+                            qk_next[t] = jq + 1;
+                            progress = true;
+                        }
+                        const int jp = pv_next[t];
+                        if (jp < n_kv && mbar_try_wait(&bars.p_ready[t], jp & 1) &&
+                            mbar_try_wait(&bars.v_full[jp % C::kStages], (jp / C::kStages) & 1)) {
+                            tc_fence_after();
+                            issue_pv(t, jp % C::kStages, jp > 0);
+                            tc_commit(&bars.pv_done[t]);
+                            pv_next[t] = jp + 1;
+                            progress = true;
+                        }
+                    }
+                    while (k_rel < min(qk_next[0], qk_next[1])) {
+                        tc_commit(&bars.k_empty[k_rel % C::kStages]);
+                        ++k_rel;
+                    }
+                    while (v_rel < min(pv_next[0], pv_next[1])) {
+                        tc_commit(&bars.v_empty[v_rel % C::kStages]);
+                        ++v_rel;
+                    }
+                    if (progress) {
+                        t_idle = 0;
+                    } else if ((++spins & 63u) == 0) {   // bounded: give up after kWaitLimitNs idle
+                        if (*abort_flag) ok = false;
+                        const uint64_t now = globaltimer_ns();
+                        if (t_idle == 0) t_idle = now;
+                        else if (now - t_idle > kWaitLimitNs) {
+                            *abort_flag = 1;
+                            record_status(-7 /* ATTN_ERR_DEVICE_TIMEOUT */);
+                            ok = false;
+                        }
+                    }
+                }
+            } else {
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j % C::kStages;
                 const uint32_t ph = (j / C::kStages) & 1;
@@ -239,6 +324,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 tc_commit(&bars.v_empty[st]);
             }
+            }
             // o_final fires when every MMA above has completed (also on the abort path,
             // so that TMEM is quiescent before it is freed)
             tc_commit(bars.o_final);
@@ -246,116 +332,162 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax warpgroups
-        const int t = warp >> 2;                        // query tile of this warpgroup
-        const int r = threadIdx.x & 127;                // row inside the tile = TMEM lane
+        // ------------------------------------------------------------ softmax warps
+        constexpr int kHalf = kTileN / 2;                // S columns per warp
+        const int t = warp >> 3;                         // query tile
+        const int hf = (warp >> 2) & 1;                  // which half of the S columns
+        const int r = ((warp & 3) << 5) | static_cast<int>(lane_id());   // row in the tile
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem_base + lane_off + C::kColS0 + t * 128;
-        const uint32_t tO = tmem_base + lane_off + C::kColO0 + t * D;
+        const uint32_t tSh = tS + hf * kHalf;            // this warp's S columns
+        const uint32_t tPh = (C::kSepP ? tmem_base + lane_off + C::kColP0 + t * 64 : tS) + hf * (kHalf / 2);
+        const uint32_t tOh = tmem_base + lane_off + C::kColO0 + t * D + hf * (D / 2);
+        float* xchg = reinterpret_cast<float*>(smem + C::kXchgOff);
+        auto xslot = [&](int buf, int half) { return xchg + ((buf * 2 + t) * 2 + half) * kTileM + r; };
         const int b = bh / H;
+        const int col0 = hf * kHalf;
         float m_run = -INFINITY;   // running max, log2 units (scale folded in)
-        float l_run = 0.f;
+        float l_run = 0.f;         // running sum over this warp's half of the columns
         bool ok = true;
+        // publish v in slot `buf` and read the partner half's value once both are in
+        auto exchange = [&](float v, int buf, uint32_t phase, float* other) -> bool {
+            *xslot(buf, hf) = v;
+            __threadfence_block();
+            tc_fence_before();   // this warp's TMEM reads of S precede the partner's P writes
+            __syncwarp();
+            if (lane_id() == 0) mbar_arrive(&bars.xchg[t]);
+            if (!mbar_wait(&bars.xchg[t], phase, abort_flag)) return false;
+            tc_fence_after();
+            *other = *xslot(buf, hf ^ 1);
+            return true;
+        };
 
         for (int j = 0; j < n_kv; ++j) {
             ok = mbar_wait(&bars.s_full[t], j & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            float s[kTileN];
-            {
-                uint32_t u[kTileN];
-                tmem_ld128_wait(tS, u);
-#pragma unroll
-                for (int i = 0; i < kTileN; ++i) s[i] = __uint_as_float(u[i]);
-            }
             const int kv0 = j * kTileN;
             const int valid = S - kv0;   // keys of this tile that exist
-            float m_tile;
-            if constexpr (kHasBias) {
-                const float* kb = key_bias + static_cast<size_t>(b) * S + kv0;
-#pragma unroll
-                for (int i = 0; i < kTileN; ++i) {
-                    const float bias = (i < valid) ? __ldg(kb + i) : -INFINITY;
-                    s[i] = (bias == -INFINITY) ? -INFINITY : fmaf(s[i], scale_log2, bias * kLog2e);
+            const bool full_tile = !kHasBias && valid >= kTileN;
+            const float* kb = nullptr;
+            if constexpr (kHasBias) kb = key_bias + static_cast<size_t>(b) * S + kv0;
+            // score of tile column i in log2 units (scale folded in), -inf where masked;
+            // only used on masked tiles (bias or a ragged last tile)
+            auto masked_score = [&](float sv, int i) -> float {
+                if (i >= valid) return -INFINITY;
+                if constexpr (kHasBias) {
+                    const float bias = __ldg(kb + i);
+                    return bias == -INFINITY ? -INFINITY : fmaf(sv, scale_log2, bias * kLog2e);
+                } else {
+                    return sv * scale_log2;
                 }
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int i = 0; i < kTileN; i += 4) {
-                    mx[0] = fmaxf(mx[0], s[i]);
-                    mx[1] = fmaxf(mx[1], s[i + 1]);
-                    mx[2] = fmaxf(mx[2], s[i + 2]);
-                    mx[3] = fmaxf(mx[3], s[i + 3]);
-                }
-                m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            } else {
-                if (valid < kTileN) {
-#pragma unroll
-                    for (int i = 0; i < kTileN; ++i)
-                        if (i >= valid) s[i] = -INFINITY;
-                }
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int i = 0; i < kTileN; i += 4) {
-                    mx[0] = fmaxf(mx[0], s[i]);
-                    mx[1] = fmaxf(mx[1], s[i + 1]);
-                    mx[2] = fmaxf(mx[2], s[i + 2]);
-                    mx[3] = fmaxf(mx[3], s[i + 3]);
-                }
-                m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
+            };
+            uint32_t u[kHalf];
+            tmem_ld64_wait(tSh, u);
+            if constexpr (C::kSepP) {   // S_t may be overwritten by the next QK from here on
+                tc_fence_before();
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(&bars.s_free[t]);
             }
+            float m_half;
+            if (full_tile) {
+                float mx[4] = {__uint_as_float(u[0]), __uint_as_float(u[1]), __uint_as_float(u[2]),
+                               __uint_as_float(u[3])};
+#pragma unroll
+                for (int i = 4; i < kHalf; i += 8) {
+                    mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+                    mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
+                    mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
+                    mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
+                }
+                m_half = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
+            } else {
+#pragma unroll
+                for (int i = 0; i < kHalf; ++i) u[i] = __float_as_uint(masked_score(__uint_as_float(u[i]), col0 + i));
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(u[i]));
+                m_half = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            }
+            float m_other;
+            ok = exchange(m_half, j & 1, j & 1, &m_other);
+            if (!ok) break;
+            const float m_tile = fmaxf(m_half, m_other);
             const bool upd = m_tile > m_run + kRescaleThreshold;
             const float m_next = upd ? m_tile : m_run;
             const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
             const float alpha = upd ? ex2_approx(m_run - m_use) : 1.f;
-            // P = exp2(s * scale_log2 - m), row sum in fp32
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // P = 2^(score - m) as bf16 pairs, 16 words at a time; row sum in fp32
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < kTileN; ++i) {
-                float p;
-                if constexpr (kHasBias) p = ex2_approx(s[i] - m_use);
-                else p = ex2_approx(fmaf(s[i], scale_log2, -m_use));
-                s[i] = p;
-                ls[i & 3] += p;
+            for (int c = 0; c < kHalf / 32; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int kk = c * 16 + k;   // column pair index in this half
+                    const float2 sv = make_float2(__uint_as_float(u[2 * kk]), __uint_as_float(u[2 * kk + 1]));
+                    float2 pv;
+                    if (full_tile) {
+                        const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
+                                                    make_float2(-m_use, -m_use));
+                        if ((kk & 7) < kPolyEighths) pv = exp2_poly2(x);
+                        else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    } else {
+                        pv = make_float2(ex2_approx(sv.x - m_use), ex2_approx(sv.y - m_use));
+                    }
+                    if (k & 1) acc1 = __fadd2_rn(acc1, pv);
+                    else acc0 = __fadd2_rn(acc0, pv);
+                    pk[k] = pack_bf16x2(pv.x, pv.y);
+                }
+                // With separate P columns, P_t and O_t are free only once PV_t of the
+                // previous tile has completed (with P over S, s_full already implied it).
+                if constexpr (C::kSepP) {
+                    if (c == 0 && j > 0) {
+                        ok = mbar_wait(&bars.pv_done[t], (j - 1) & 1, abort_flag);
+                        tc_fence_after();
+                    }
+                }
+                // Both halves read their S columns before the exchange above, so P columns
+                // that overlap the first half's S columns are free to write.
+                tmem_st16(tPh + c * 16, pk);
             }
-            l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+            if (!ok) break;
+            l_run = l_run * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
             m_run = m_next;
-            // rescale this row of O (only if some row of the warp moved its max)
+            // rescale this warp's half of the O row (only if some row of the warp moved its max)
             if (j > 0 && __any_sync(0xffffffffu, upd)) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t u[32];
-                    tmem_ld32_wait(tO + c * 32, u);
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32_wait(tOh + c * 32, w);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-                    tmem_st32(tO + c * 32, u);
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                    tmem_st32(tOh + c * 32, w);
                 }
-            }
-            // P (bf16 pairs) over the first 64 columns of S_t
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t u[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) u[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
-                tmem_st32(tS + c * 32, u);
             }
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars.p_ready[t]);
+            __syncwarp();
+            if (lane_id() == 0) mbar_arrive(&bars.p_ready[t]);
         }
+        // full row sum = both halves
+        float l_other = 0.f;
+        if (ok) ok = exchange(l_run, n_kv & 1, n_kv & 1, &l_other);
         if (ok) ok = mbar_wait(bars.o_final, 0, abort_flag);
         if (ok) {
             tc_fence_after();
+            const float l_tot = l_run + l_other;
             const int row = row0 + t * kTileM + r;
-            const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-            uint16_t* orow = out + (static_cast<size_t>(bh) * S + row) * D;
+            const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+            uint16_t* orow = out + (static_cast<size_t>(bh) * S + row) * D + hf * (D / 2);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t u[32];
-                tmem_ld32_wait(tO + c * 32, u);
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t w[32];
+                tmem_ld32_wait(tOh + c * 32, w);
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+                    pk[i] = pack_bf16x2(__uint_as_float(w[2 * i]) * inv_l, __uint_as_float(w[2 * i + 1]) * inv_l);
                 if (row < S) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll

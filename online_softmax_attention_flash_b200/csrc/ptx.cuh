@@ -331,6 +331,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// max of three fp32 values (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x on the FMA pipe, for two values at once (packed f32x2 arithmetic).
+// Range reduction x = n + f with n = round(x), f in [-1/2, 1/2] (Cody-Waite style,
+// n obtained by adding and subtracting 1.5 * 2^23); 2^f from a degree-3 minimax
+// polynomial fitted for this library by the Remez exchange algorithm on
+// [-1/2, 1/2] (max relative error 7.5e-5); 2^n enters through the exponent
+// field. Inputs are clamped at -125 so that the exponent never underflows.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+    constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 j = __fadd2_rn(x, make_float2(kShift, kShift));
+    const float2 n = __fadd2_rn(j, make_float2(-kShift, -kShift));
+    const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+    float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+    p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
+}
+
 // Two fp32 -> two E4M3FN (round-to-nearest-even, saturating); element `lo` in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3x2_f32(float lo, float hi) {
     uint16_t r;
