@@ -101,6 +101,8 @@ ATTN_API size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx
  *   out       : [B, Hq, 1, D] bf16
  *   Hq == Hkv * num_kv_groups; query head h reads kv head h / num_kv_groups.
  *   D in {128, 256, 512}; S_ctx >= 1 (no multiple-of-128 requirement).
+ *   num_kv_groups in {1, 2, 4, 8}; D == 512 allows at most 4 (else
+ *   ATTN_ERR_UNSUPPORTED).
  *   workspace : device buffer of at least attn_gqa_decode_workspace_size(...)
  *               bytes, 16-byte aligned, owned by the caller; its contents on
  *               entry do not matter. Calls that share one workspace must not

@@ -39,10 +39,15 @@ def test_head_dims_and_groups(D, G):
     Hkv = 2
     case = syn.decode_case(3, Hkv * G, Hkv, 700, D, seed=10 * D + G, softmax_scale=D ** -0.5,
                            min_len=1, max_len=700)
+    if D == 512 and G == 8:   # outside the supported set: rejected before any launch
+        with pytest.raises(B.AttnError) as exc:
+            _run(case)
+        assert exc.value.status == -3
+        return
     assert_bf16_parity(_run(case), _oracle(case), 2, f"D={D} G={G}")
 
 
-@pytest.mark.parametrize("S_ctx", [1, 31, 32, 33, 255, 256, 257, 1000])
+@pytest.mark.parametrize("S_ctx", [1, 7, 8, 9, 31, 32, 33, 255, 256, 257, 511, 512, 513, 1000])
 def test_ragged_context_without_mask(S_ctx):
     case = syn.decode_case(2, 4, 2, S_ctx, 256, seed=S_ctx, lengths=[S_ctx, S_ctx])
     assert_bf16_parity(_run(case, use_mask=False), _oracle(case, use_mask=False), 2,
