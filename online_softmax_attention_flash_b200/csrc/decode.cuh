@@ -67,7 +67,7 @@ struct Cfg {
     static constexpr int kScrFloats = kMaxGroups * kSubKeys + kMaxGroups;
     static constexpr int kListOff = kScrOff + kWarps * kScrFloats * 4;      // live sub-tiles
     static constexpr int kBarOff = kListOff + (kSubTiles + 4) * 4;
-    static constexpr int kMiscOff = kBarOff + kWarps * kStages * 8;
+    static constexpr int kMiscOff = kBarOff + kWarps * kStages * 2 * 8;   // K and V barrier per stage
     static constexpr int kSmemBytes = kMiscOff + 16;
 };
 
@@ -140,13 +140,13 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     const int key0 = split * kSplitKeys;
     const size_t kv_base = (static_cast<size_t>(b) * Hkv + g) * S_ctx;
     float* scr = reinterpret_cast<float*>(smem + C::kScrOff) + warp * C::kScrFloats;
-    uint64_t* my_full = full + warp * C::kStages;
+    uint64_t* my_full = full + warp * C::kStages * 2;   // [stage][K, V]
     uint8_t* my_ring = smem + C::kRingOff + warp * C::kStages * C::kStageBytes;
 
     // the combine kernel may be scheduled now; it waits for this grid's completion itself
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
-        for (int s = 0; s < kWarps * C::kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < kWarps * C::kStages * 2; ++s) mbar_init(&full[s], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -177,19 +177,25 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     // this warp's share: live sub-tiles warp, warp + 4, ...
     const int my_count = n_live > warp ? (n_live - warp + kWarps - 1) / kWarps : 0;
 
-    auto issue = [&](int i) {   // i-th sub-tile of this warp -> its stage i % kStages
+    // K and V rows of this warp's i-th sub-tile go to stage i % kStages, each half with
+    // its own barrier, so that K can be refilled as soon as the scores are computed
+    int issued[2] = {0, 0};   // sub-tiles whose K / V copy this warp has started (lane 0)
+    auto issue_half = [&](int i, int which) {
+        issued[which] = i + 1;
         const int st = i % C::kStages;
         const int sub = live[warp + i * kWarps];
         const int kk0 = key0 + sub * kSubKeys;
         const int rows = min(kSubKeys, S_ctx - kk0);
         const uint32_t bytes = static_cast<uint32_t>(rows) * C::kRowBytes;
-        uint8_t* dst = my_ring + st * C::kStageBytes;
-        mbar_arrive_expect_tx(&my_full[st], 2 * bytes);
-        bulk_load(dst, k + (kv_base + kk0) * D, bytes, &my_full[st]);
-        bulk_load(dst + C::kSubBytes, v + (kv_base + kk0) * D, bytes, &my_full[st]);
+        uint8_t* dst = my_ring + st * C::kStageBytes + which * C::kSubBytes;
+        mbar_arrive_expect_tx(&my_full[2 * st + which], bytes);
+        bulk_load(dst, (which ? v : k) + (kv_base + kk0) * D, bytes, &my_full[2 * st + which]);
     };
     if (lane == 0)
-        for (int i = 0; i < my_count && i < C::kStages; ++i) issue(i);
+        for (int i = 0; i < my_count && i < C::kStages; ++i) {
+            issue_half(i, 0);
+            issue_half(i, 1);
+        }
 
     // q of the G heads: this lane's slice [lane*EPL, lane*EPL + EPL), pre-scaled to log2 units
     float qr[G][C::kEPL];
@@ -222,7 +228,7 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
         const int sub = live[warp + i * kWarps];
         const int kk0 = key0 + sub * kSubKeys;
         const int rows = min(kSubKeys, S_ctx - kk0);
-        ok = mbar_wait(&my_full[st], (i / C::kStages) & 1, abort_flag);
+        ok = mbar_wait(&my_full[2 * st], (i / C::kStages) & 1, abort_flag);
         if (!ok) break;
         const uint8_t* Ks = my_ring + st * C::kStageBytes;
         const uint8_t* Vs = Ks + C::kSubBytes;
@@ -251,6 +257,10 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
                 for (int hh = 0; hh < kHeadsPerPass; ++hh) part[hh * kSubKeys + kk] = acc[hh];
             }
             transpose_reduce<kN>(part, lane);
+            if (pass == kPasses - 1) {   // every lane is done reading K of this stage
+                __syncwarp();
+                if (lane == 0 && i + C::kStages < my_count) issue_half(i + C::kStages, 0);
+            }
             // lane now holds the score of value idx = lane / kBase: head hh = idx / 8, key kk = idx % 8
             const int idx = lane / kBase;
             const int hh_me = idx / kSubKeys, kk_me = idx % kSubKeys;
@@ -290,6 +300,12 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
 #pragma unroll
                 for (int e = 0; e < C::kEPL; ++e) o[h][e] *= a;
             }
+            if (pass == 0) {
+                if (!mbar_wait(&my_full[2 * st + 1], (i / C::kStages) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+            }
             // ---- O += P V for this pass's heads (rows past S_ctx hold stale data: skipped)
 #pragma unroll
             for (int kk = 0; kk < kSubKeys; ++kk) {
@@ -313,11 +329,14 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
             }
             __syncwarp();   // scratch is rewritten by the next pass / sub-tile
         }
-        // this stage is consumed: refill it with the sub-tile kStages ahead
-        if (lane == 0 && i + C::kStages < my_count) issue(i + C::kStages);
+        if (!ok) break;
+        // V of this stage is consumed: refill it with the sub-tile kStages ahead
+        if (lane == 0 && i + C::kStages < my_count) issue_half(i + C::kStages, 1);
     }
-    if (!ok && lane == 0) {
-        for (int i = 0; i < my_count && i < C::kStages; ++i) mbar_wait_drain(&my_full[i % C::kStages], 0);
+    if (!ok && lane == 0) {   // let every copy this warp started land before the CTA exits
+        for (int which = 0; which < 2; ++which)
+            for (int i = max(0, issued[which] - C::kStages); i < issued[which]; ++i)
+                mbar_wait_drain(&my_full[2 * (i % C::kStages) + which], (i / C::kStages) & 1);
     }
     __syncthreads();   // every warp is done with its ring: reuse it for the merge
 
