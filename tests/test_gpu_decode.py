@@ -98,3 +98,34 @@ def test_fully_masked_row_is_zero():
     case.attn_mask.fill_(float("-inf"))
     out = _run(case).cpu()
     assert torch.count_nonzero(out) == 0
+
+
+@pytest.mark.parametrize("W", [64, 500, 1024])
+def test_sliding_window_mask(W):
+    """Sliding-window layers (the decode page's windowed-KV follow-on) as an additive
+    mask: only the last W positions before each length are kept; the kernel reads only
+    the 8-key groups that hold them."""
+    case = syn.decode_case(4, 8, 4, 4096, 256, seed=W, softmax_scale=256 ** -0.5)
+    for b in range(4):
+        L = int(case.lengths[b])
+        case.attn_mask[b, ..., :max(0, L - W)] = float("-inf")
+    assert_bf16_parity(_run(case), _oracle(case), 2, f"window {W}")
+
+
+def test_head_dim_512_gemma_global_layer_shape():
+    """Gemma global layers (decode page: head_dim 512), 2 Q heads per KV head."""
+    case = syn.decode_case(2, 16, 8, 2048, 512, seed=512, softmax_scale=1.0, min_len=1)
+    assert_bf16_parity(_run(case), _oracle(case), 2, "D=512")
+
+
+def test_one_workspace_reused_across_calls_with_different_split_counts():
+    """The workspace's arrival counters return to zero after every call, so one
+    zeroed workspace serves calls of any size in turn."""
+    need = max(B.attn_gqa_decode_workspace_size(2, 8, 4, S, 256) for S in (4096, 700, 1, 2600))
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    for S in (4096, 700, 1, 2600, 4096):
+        case = syn.decode_case(2, 8, 4, S, 256, seed=S, softmax_scale=1 / 16, min_len=1, max_len=S)
+        q, k, v, m = (t.to(DEV) for t in (case.q, case.k, case.v, case.attn_mask))
+        out = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups, workspace=ws)
+        assert B.attn_check() == 0
+        assert_bf16_parity(out, _oracle(case), 2, f"reuse S_ctx={S}")

@@ -104,3 +104,25 @@ def test_batch_independence_bitwise():
 def test_deterministic_repeat():
     case = syn.encoder_case(1, 4, 700, 64, seed=98)
     assert torch.equal(_run(case).cpu(), _run(case).cpu())
+
+
+def test_long_sequence_8192_tokens_sampled_rows():
+    """V-JEPA2's native 64-frame clip is 8192 tokens; the V-JEPA2 page's kernels could not
+    run it (their cross-section combine). Online softmax has no section limit."""
+    case = syn.encoder_case(1, 2, 8192, 64, seed=8192, softmax_scale=0.125)
+    out = _run(case)
+    rows = np.sort(np.random.default_rng(1).choice(8192, 256, replace=False))
+    ref = _oracle(case, rows=rows)
+    assert_bf16_parity(out[:, :, torch.from_numpy(rows).to(out.device)], ref, 2, "S=8192")
+
+
+@pytest.mark.parametrize("L", [128, 512, 1024])
+def test_gte_shapes_right_padded_batches(L):
+    """gte encoders: head_dim 64, 16 heads, right-padded batches of ragged lengths
+    (gte page "Accuracy": 6 tokens up to the padded length)."""
+    lens = [L, 6, L // 2 + 3, L - 1]
+    case = syn.encoder_case(4, 16, L, 64, seed=L, softmax_scale=0.125, pad_lengths=lens)
+    out = _run(case)
+    ref = _oracle(case)
+    # rows of padded positions also attend to the valid keys; all rows are compared
+    assert_bf16_parity(out, ref, 2, f"gte L={L}")
