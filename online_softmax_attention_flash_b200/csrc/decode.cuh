@@ -238,23 +238,22 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
             float part[32];
 #pragma unroll
             for (int kk = 0; kk < kSubKeys; ++kk) {
-                float acc[kHeadsPerPass];
+                float2 acc[kHeadsPerPass];   // even / odd elements, packed fp32x2 FMAs
 #pragma unroll
-                for (int hh = 0; hh < kHeadsPerPass; ++hh) acc[hh] = 0.f;
+                for (int hh = 0; hh < kHeadsPerPass; ++hh) acc[hh] = make_float2(0.f, 0.f);
                 uint32_t ws[C::kEPL / 2];
                 load_bf16_words<C::kEPL>(Ks + kk * C::kRowBytes + lane * C::kEPL * 2, ws);
 #pragma unroll
                 for (int i2 = 0; i2 < C::kEPL / 2; ++i2) {
-                    const float k0 = bf16_lo(ws[i2]), k1 = bf16_hi(ws[i2]);
+                    const float2 kv = make_float2(bf16_lo(ws[i2]), bf16_hi(ws[i2]));
 #pragma unroll
                     for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                         const int h = pass * kHeadsPerPass + hh;
-                        acc[hh] = fmaf(qr[h][2 * i2], k0, acc[hh]);
-                        acc[hh] = fmaf(qr[h][2 * i2 + 1], k1, acc[hh]);
+                        acc[hh] = __ffma2_rn(make_float2(qr[h][2 * i2], qr[h][2 * i2 + 1]), kv, acc[hh]);
                     }
                 }
 #pragma unroll
-                for (int hh = 0; hh < kHeadsPerPass; ++hh) part[hh * kSubKeys + kk] = acc[hh];
+                for (int hh = 0; hh < kHeadsPerPass; ++hh) part[hh * kSubKeys + kk] = acc[hh].x + acc[hh].y;
             }
             transpose_reduce<kN>(part, lane);
             if (pass == kPasses - 1) {   // every lane is done reading K of this stage
@@ -288,7 +287,9 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
             if ((lane % kBase) == 0) scr[hh_me * kSubKeys + kk_me] = p;
             if ((lane % kBase) == 0 && kk_me == 0) scr[kMaxGroups * kSubKeys + hh_me] = alpha;
             __syncwarp();
-            // every lane updates the running state of the heads of this pass
+            // every lane updates the running state of the heads of this pass; O is rescaled
+            // only if some head's max moved (after the first sub-tiles it rarely does)
+            const bool any_moved = __any_sync(0xffffffffu, m_new != m_old);
 #pragma unroll
             for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                 const int h = pass * kHeadsPerPass + hh;
@@ -297,8 +298,14 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
                 const float sum = __shfl_sync(0xffffffffu, ps, hh * kSubKeys * kBase);
                 l_run[h] = l_run[h] * a + sum;
                 m_run[h] = mn;
+                if (any_moved) {
 #pragma unroll
-                for (int e = 0; e < C::kEPL; ++e) o[h][e] *= a;
+                    for (int e = 0; e < C::kEPL; e += 2) {
+                        const float2 r = __fmul2_rn(make_float2(o[h][e], o[h][e + 1]), make_float2(a, a));
+                        o[h][e] = r.x;
+                        o[h][e + 1] = r.y;
+                    }
+                }
             }
             if (pass == 0) {
                 if (!mbar_wait(&my_full[2 * st + 1], (i / C::kStages) & 1, abort_flag)) {
@@ -317,12 +324,14 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
                     for (int hh = 0; hh < kHeadsPerPass; ++hh) pk[hh] = scr[hh * kSubKeys + kk];
 #pragma unroll
                     for (int i2 = 0; i2 < C::kEPL / 2; ++i2) {
-                        const float v0 = bf16_lo(ws[i2]), v1 = bf16_hi(ws[i2]);
+                        const float2 vv = make_float2(bf16_lo(ws[i2]), bf16_hi(ws[i2]));
 #pragma unroll
                         for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                             const int h = pass * kHeadsPerPass + hh;
-                            o[h][2 * i2] = fmaf(pk[hh], v0, o[h][2 * i2]);
-                            o[h][2 * i2 + 1] = fmaf(pk[hh], v1, o[h][2 * i2 + 1]);
+                            const float2 r = __ffma2_rn(make_float2(pk[hh], pk[hh]), vv,
+                                                        make_float2(o[h][2 * i2], o[h][2 * i2 + 1]));
+                            o[h][2 * i2] = r.x;
+                            o[h][2 * i2 + 1] = r.y;
                         }
                     }
                 }
