@@ -58,9 +58,8 @@ int launch_encoder(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint
     if ((rc = attn::encode_map_3d_bf16(&tv, v, D, rows, heads, 64, kTileN))) return rc;
     dim3 grid((S + kRowsPerCta - 1) / kRowsPerCta, static_cast<unsigned>(heads));
     const float scale_log2 = scale * kLog2e;
-    kernel<<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, out, key_bias, H, S,
-                                                           scale_log2);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return attn::launch_pdl(kernel, grid, dim3(kThreads), Cfg<D>::kSmemBytes, stream, tq, tk, tv, out,
+                            key_bias, H, S, scale_log2);
 }
 
 // Scratch for attn_gqa_decode_noalloc: reserved statically on every device that

@@ -29,6 +29,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "tmap.cuh"
 
 namespace attn {
 namespace dec {
@@ -144,12 +145,14 @@ decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     uint8_t* my_ring = smem + C::kRingOff + warp * C::kStages * C::kStageBytes;
 
     // the combine kernel may be scheduled now; it waits for this grid's completion itself
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_launch_dependents();
     if (tid == 0) {
         for (int s = 0; s < kWarps * C::kStages * 2; ++s) mbar_init(&full[s], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // the previous kernel on the stream may still be reading this workspace: wait for it
+    pdl_wait_predecessor();
     // additive mask of this split in log2 units (-inf past S_ctx); live 8-key sub-tiles
     for (int i = tid; i < kSplitKeys; i += kThreads) {
         const int key = key0 + i;
@@ -396,7 +399,7 @@ decode_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ 
                       const float* __restrict__ ws_l, uint16_t* __restrict__ out, int n_split) {
     // launched as a programmatic dependent of the split kernel: wait until its writes
     // to the workspace are complete and visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait_predecessor();
     const size_t row = blockIdx.x;   // b * Hq + h
     const float* m = ws_m + row * n_split;
     const float* l = ws_l + row * n_split;
@@ -443,24 +446,12 @@ int launch_dg(const uint16_t* q, const uint16_t* k, const uint16_t* v, const flo
     }
     const int n_split = num_splits(S_ctx);
     dim3 grid(n_split, Hkv, B);
-    decode_split_kernel<D, G><<<grid, C::kThreads, C::kSmemBytes, stream>>>(
-        q, k, v, mask, ws_o, ws_m, ws_l, Hkv, S_ctx, scale * kLog2e);
-    if (cudaGetLastError() != cudaSuccess) return -6;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(B * Hkv * G);
-    cfg.blockDim = dim3(D / 4);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, static_cast<const float*>(ws_o),
-                           static_cast<const float*>(ws_m), static_cast<const float*>(ws_l), out,
-                           n_split) != cudaSuccess)
+    if (launch_pdl(decode_split_kernel<D, G>, grid, dim3(C::kThreads), C::kSmemBytes, stream, q, k,
+                   v, mask, ws_o, ws_m, ws_l, Hkv, S_ctx, scale * kLog2e))
         return -6;
-    return 0;
+    return launch_pdl(decode_combine_kernel<D>, dim3(B * Hkv * G), dim3(D / 4), 0, stream,
+                      static_cast<const float*>(ws_o), static_cast<const float*>(ws_m),
+                      static_cast<const float*>(ws_l), out, n_split);
 }
 
 template <int D>

@@ -38,12 +38,12 @@ constexpr int kSoftmaxWarps = 16;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
-#ifndef ATTN_ENC_POLY_EIGHTHS
-#define ATTN_ENC_POLY_EIGHTHS 3
-#endif
 // Of every 8 column pairs of an unmasked S tile, this many take 2^x from the FMA-pipe
-// polynomial instead of the MUFU ex2 unit (which alone caps D=64 at half the MMA rate).
-constexpr int kPolyEighths = ATTN_ENC_POLY_EIGHTHS;
+// polynomial instead of the MUFU ex2 unit. At D = 64 the exponentials are as many per
+// MMA flop as MUFU can barely sustain, so a share moves to the FMA pipe; at D = 128
+// MUFU has room and the polynomial only costs issue slots.
+template <int D>
+__host__ __device__ constexpr int poly_eighths() { return D == 64 ? 2 : 0; }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -157,6 +157,9 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // set-up done: let the next kernel on the stream start, then wait for the previous one
+    pdl_launch_dependents();
+    pdl_wait_predecessor();
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
@@ -430,7 +433,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (full_tile) {
                         const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
                                                     make_float2(-m_use, -m_use));
-                        if ((kk & 7) < kPolyEighths) pv = exp2_poly2(x);
+                        if ((kk & 7) < poly_eighths<D>()) pv = exp2_poly2(x);
                         else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     } else {
                         pv = make_float2(ex2_approx(sv.x - m_use), ex2_approx(sv.y - m_use));

@@ -139,6 +139,8 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+    pdl_wait_predecessor();
 
     if (warp == kProducerWarp) {
         // ---------------------------------------------------------------- producer
@@ -470,8 +472,7 @@ inline int launch(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_ca
     prm.c_qk = k_scale * softmax_scale * kLog2e;
     prm.v_scale = v_scale;
     dim3 grid((Sq + kTileM - 1) / kTileM, Hq);
-    paged_history_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, prm);
-    return cudaGetLastError() == cudaSuccess ? 0 : -6;
+    return launch_pdl(paged_history_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, prm);
 }
 
 }  // namespace paged

@@ -53,4 +53,22 @@ inline int encode_map_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uin
     return encode_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, d0, d1, d2, box0, box1);
 }
 
+// Launch `kernel` on `stream` with programmatic stream serialization (the kernel
+// overlaps its set-up with the previous kernel's tail; see pdl_wait_predecessor).
+template <typename Kernel, typename... Args>
+inline int launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? 0 : -6;
+}
+
 }  // namespace attn
