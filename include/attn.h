@@ -82,7 +82,9 @@ ATTN_API int attn_encoder_fwd(const uint16_t* q, const uint16_t* k, const uint16
 
 /*
  * attn_gqa_decode_workspace_size -- bytes of device workspace attn_gqa_decode
- * needs for these sizes (the split-KV partial results). 0 for invalid sizes.
+ * needs for these sizes: the per-batch lists of live 8-key sub-tiles with their
+ * mask values, and the partial results of the key-sequence split (one per warp
+ * and (batch, kv head) pair it covers). 0 for invalid sizes.
  */
 ATTN_API size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx, int D);
 
@@ -102,7 +104,8 @@ ATTN_API size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx
  *   Hq == Hkv * num_kv_groups; query head h reads kv head h / num_kv_groups.
  *   D in {128, 256, 512}; S_ctx >= 1 (no multiple-of-128 requirement).
  *   num_kv_groups in {1, 2, 4, 8}; D == 512 allows at most 4 (else
- *   ATTN_ERR_UNSUPPORTED).
+ *   ATTN_ERR_UNSUPPORTED). B * Hkv <= 65535 and B * Hkv * ceil(S_ctx / 8) < 2^30
+ *   (else ATTN_ERR_UNSUPPORTED).
  *   workspace : device buffer of at least attn_gqa_decode_workspace_size(...)
  *               bytes, 16-byte aligned, owned by the caller; its contents on
  *               entry do not matter. Calls that share one workspace must not
@@ -146,7 +149,7 @@ ATTN_API int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_
  * Errors: as attn_gqa_decode; ATTN_ERR_WORKSPACE when the sizes exceed the
  * scratch; ATTN_ERR_CUDA if the address look-up fails.
  */
-#define ATTN_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+#define ATTN_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 ATTN_API int attn_gqa_decode_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      const float* attn_mask, uint16_t* out,
                                      int B, int Hq, int Hkv, int num_kv_groups, int S_ctx, int D,

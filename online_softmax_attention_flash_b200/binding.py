@@ -157,7 +157,7 @@ def attn_gqa_decode(q, k, v, attn_mask, softmax_scale: float, num_kv_groups: int
     return out
 
 
-NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024   # ATTN_NOALLOC_SCRATCH_BYTES in include/attn.h
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # ATTN_NOALLOC_SCRATCH_BYTES in include/attn.h
 
 
 def attn_gqa_decode_noalloc(q, k, v, attn_mask, softmax_scale: float, num_kv_groups: int,

@@ -139,7 +139,7 @@ int attn_encoder_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, ui
 
 size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx, int D) {
     if (B < 1 || Hq < 1 || Hkv < 1 || S_ctx < 1 || D < 1 || Hq % Hkv) return 0;
-    return attn::dec::workspace_bytes(B, Hq, S_ctx, D);
+    return attn::dec::workspace_bytes(B, Hq, Hkv, S_ctx, D);
 }
 
 int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -151,10 +151,11 @@ int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     if (Hq != Hkv * num_kv_groups || !scale_ok(softmax_scale)) return ATTN_ERR_SHAPE;
     if (D != 128 && D != 256 && D != 512) return ATTN_ERR_UNSUPPORTED;
     if (num_kv_groups > attn::dec::kMaxGroups) return ATTN_ERR_UNSUPPORTED;
-    if (static_cast<int64_t>(B) * Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * Hkv > 65535 || !attn::dec::items_fit(B, Hkv, S_ctx))
+        return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_ALIGN;
     if (attn_mask && (reinterpret_cast<uintptr_t>(attn_mask) & 15u)) return ATTN_ERR_ALIGN;
-    const size_t need = attn::dec::workspace_bytes(B, Hq, S_ctx, D);
+    const size_t need = attn::dec::workspace_bytes(B, Hq, Hkv, S_ctx, D);
     if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
     return attn::dec::launch(q, k, v, attn_mask, out, B, Hq, Hkv, num_kv_groups, S_ctx, D,
@@ -166,7 +167,7 @@ int attn_gqa_decode_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t
                             int num_kv_groups, int S_ctx, int D, float softmax_scale,
                             void* stream) {
     if (B < 1 || Hq < 1 || Hkv < 1 || S_ctx < 1 || Hq % Hkv) return ATTN_ERR_SHAPE;
-    const size_t need = attn::dec::workspace_bytes(B, Hq, S_ctx, D);
+    const size_t need = attn::dec::workspace_bytes(B, Hq, Hkv, S_ctx, D);
     if (need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
     void* scratch = nullptr;
     const int rc = noalloc_scratch(&scratch);

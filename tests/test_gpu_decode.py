@@ -119,8 +119,8 @@ def test_head_dim_512_gemma_global_layer_shape():
 
 
 def test_one_workspace_reused_across_calls_with_different_split_counts():
-    """The workspace's arrival counters return to zero after every call, so one
-    zeroed workspace serves calls of any size in turn."""
+    """One workspace serves calls of any size in turn: every call rebuilds the live
+    lists and partials it reads, whatever the previous call left there."""
     need = max(B.attn_gqa_decode_workspace_size(2, 8, 4, S, 256) for S in (4096, 700, 1, 2600))
     ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     for S in (4096, 700, 1, 2600, 4096):
@@ -129,3 +129,44 @@ def test_one_workspace_reused_across_calls_with_different_split_counts():
         out = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups, workspace=ws)
         assert B.attn_check() == 0
         assert_bf16_parity(out, _oracle(case), 2, f"reuse S_ctx={S}")
+
+
+def test_tiny_contexts_many_pairs_per_warp():
+    """Short, ragged contexts: each warp's slice of the live sub-tile sequence crosses
+    many (batch, kv head) pairs, and with S_ctx = 16 there are fewer sub-tiles than
+    warps (most warps idle)."""
+    for B_, S, seed in ((64, 64, 71), (2, 16, 72)):
+        case = syn.decode_case(B_, 16, 8, S, 256, seed=seed, softmax_scale=1 / 16, min_len=1)
+        assert_bf16_parity(_run(case), _oracle(case), 2, f"tiny contexts B={B_} S={S}")
+
+
+def test_fully_masked_batch_entries_between_live_ones():
+    """Batch entries without a live key produce zero rows and shift the numbering of
+    the following entries' partials; their neighbours must be unaffected."""
+    case = syn.decode_case(7, 8, 4, 1200, 128, seed=73, softmax_scale=128 ** -0.5, min_len=1)
+    for b in (0, 3, 4, 6):
+        case.attn_mask[b].fill_(float("-inf"))
+    out = _run(case)
+    ref = _oracle(case)
+    assert_bf16_parity(out, ref, 2, "masked entries")
+    assert torch.count_nonzero(out[[0, 3, 4, 6]].cpu()) == 0
+
+
+def test_one_long_pair_spread_over_every_warp():
+    """A single (batch, kv head) pair with 32768 keys: its live sub-tiles are split
+    over all warps of the wave, so the combine merges well over a thousand partials."""
+    case = syn.decode_case(1, 8, 1, 32768, 256, seed=74, softmax_scale=1 / 16,
+                           lengths=[32768])
+    assert_bf16_parity(_run(case), _oracle(case), 2, "one long pair")
+
+
+def test_workspace_contents_on_entry_do_not_matter():
+    case = syn.decode_case(3, 8, 2, 3000, 256, seed=75, softmax_scale=1 / 16, min_len=1)
+    q, k, v, m = (t.to(DEV) for t in (case.q, case.k, case.v, case.attn_mask))
+    need = B.attn_gqa_decode_workspace_size(3, 8, 2, 3000, 256)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bit patterns
+    out = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups, workspace=ws)
+    assert B.attn_check() == 0
+    ref = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups)
+    assert torch.equal(out.cpu(), ref.cpu())
+    assert_bf16_parity(out, _oracle(case), 2, "garbage workspace")

@@ -50,7 +50,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 def test_noalloc_rejects_sizes_beyond_the_scratch():
     lib = B.load_library()
     fake = ctypes.c_void_p(4096)   # never dereferenced: the size check comes first
-    # 64 x 64 heads x 256 splits x 512 floats is far beyond the 4 MiB scratch
+    # 64 batch entries x 8192 sub-tiles of lists alone are beyond the scratch
     st = lib.attn_gqa_decode_noalloc(fake, fake, fake, None, fake, 64, 64, 8, 8, 65536, 512,
                                      1.0, None)
     assert st == -5   # ATTN_ERR_WORKSPACE
