@@ -231,11 +231,11 @@ class DecodeWork:
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.bytes = [oracle.decode_algorithmic_bytes(c.lengths.tolist(), cfg["Hkv"], cfg["D"],
                                                       cfg["Hq"], cfg["S"]) for c in self.host]
-        self.launches_per_step = 2   # split + combine
+        self.launches_per_step = 3   # scan + stream + combine
         self.work_per_step = float(np.mean(self.bytes))
         self.flops_per_launch = self.work_per_step
         self.unit, self.bound = "GB/s", "hbm"
-        self.kernel_regex = "decode_split_kernel"
+        self.kernel_regex = "decode_stream_kernel"
         self.peak_ratio = 1.0
         self.dtype = "bf16"
         self.i = 0
@@ -489,7 +489,7 @@ def run_product(args, info):
     peaks, peak_src = load_peaks()
     per_launch_ms = total_ms / (args.steps * work.launches_per_step)
     if work.bound == "hbm":
-        # decode: one call = split + combine; achieved counts the whole call's time
+        # decode: one call = scan + stream + combine; achieved counts the whole call's time
         per_call_ms = total_ms / args.steps
         achieved = work.work_per_step / (per_call_ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])

@@ -43,7 +43,7 @@ constexpr int kThreads = 576;
 // MMA flop as MUFU can barely sustain, so a share moves to the FMA pipe; at D = 128
 // MUFU has room and the polynomial only costs issue slots.
 template <int D>
-__host__ __device__ constexpr int poly_eighths() { return D == 64 ? 2 : 0; }
+__host__ __device__ constexpr int poly_eighths() { return D == 64 ? 1 : 0; }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -246,57 +246,46 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tc_commit(&bars.k_empty[0]);
             }
             if constexpr (C::kSepP) {
-                // Issue whichever MMA is ready: QK_t(j) needs K_j and the softmax to have read
-                // S_t(j-1); PV_t(j) needs V_j and P_t(j). The two query tiles progress
-                // independently; a K / V stage is released once both tiles have used it.
-                int qk_next[kQTiles] = {1, 1}, pv_next[kQTiles] = {0, 0};
-                int k_rel = 1, v_rel = 0;
-                uint64_t t_idle = 0;
-                uint32_t spins = 0;
-                while (ok && (pv_next[0] < n_kv || pv_next[1] < n_kv)) {
-                    bool progress = false;
-#pragma unroll
-                    for (int t = 0; t < kQTiles; ++t) {
-                        const int jq = qk_next[t];
-                        if (jq < n_kv && mbar_try_wait(&bars.s_free[t], (jq - 1) & 1) &&
-                            mbar_try_wait(&bars.k_full[jq % C::kStages], (jq / C::kStages) & 1)) {
-                            tc_fence_after();
-                            issue_qk(t, jq % C::kStages);
-                            tc_commit(&bars.s_full[t]);
-                            qk_next[t] = jq + 1;
-                            progress = true;
-                        }
-                        const int jp = pv_next[t];
-                        if (jp < n_kv && mbar_try_wait(&bars.p_ready[t], jp & 1) &&
-                            mbar_try_wait(&bars.v_full[jp % C::kStages], (jp / C::kStages) & 1)) {
-                            tc_fence_after();
-                            issue_pv(t, jp % C::kStages, jp > 0);
-                            tc_commit(&bars.pv_done[t]);
-                            pv_next[t] = jp + 1;
-                            progress = true;
-                        }
+                // Fixed issue order per key tile j, the order in which the softmax warpgroups
+                // free their inputs (tile 1 runs half a key tile behind tile 0):
+                //   QK_0(j+1) once tile 0 has read S_0(j); PV_1(j-1) once P_1(j-1) is written;
+                //   QK_1(j+1) once tile 1 has read S_1(j); PV_0(j) once P_0(j) is written.
+                // Every wait is on a barrier whose producer depends only on MMAs issued
+                // earlier in this order. A K stage is released after QK_1 has used it, a V
+                // stage after PV_1.
+                auto pv = [&](int t, int j) -> bool {
+                    const int sp = j % C::kStages;
+                    if (!mbar_wait(&bars.p_ready[t], j & 1, abort_flag)) return false;
+                    if (!mbar_wait(&bars.v_full[sp], (j / C::kStages) & 1, abort_flag)) return false;
+                    tc_fence_after();
+                    issue_pv(t, sp, j > 0);
+                    tc_commit(&bars.pv_done[t]);
+                    if (t == 1) tc_commit(&bars.v_empty[sp]);
+                    return true;
+                };
+                for (int j = 0; j < n_kv && ok; ++j) {
+                    const bool more = j + 1 < n_kv;
+                    const int stn = (j + 1) % C::kStages;
+                    if (more) {
+                        ok = mbar_wait(&bars.s_free[0], j & 1, abort_flag) &&
+                             mbar_wait(&bars.k_full[stn], ((j + 1) / C::kStages) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(0, stn);
+                        tc_commit(&bars.s_full[0]);
                     }
-                    while (k_rel < min(qk_next[0], qk_next[1])) {
-                        tc_commit(&bars.k_empty[k_rel % C::kStages]);
-                        ++k_rel;
+                    if (j > 0 && !(ok = pv(1, j - 1))) break;
+                    if (more) {
+                        ok = mbar_wait(&bars.s_free[1], j & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(1, stn);
+                        tc_commit(&bars.s_full[1]);
+                        tc_commit(&bars.k_empty[stn]);
                     }
-                    while (v_rel < min(pv_next[0], pv_next[1])) {
-                        tc_commit(&bars.v_empty[v_rel % C::kStages]);
-                        ++v_rel;
-                    }
-                    if (progress) {
-                        t_idle = 0;
-                    } else if ((++spins & 63u) == 0) {   // bounded: give up after kWaitLimitNs idle
-                        if (*abort_flag) ok = false;
-                        const uint64_t now = globaltimer_ns();
-                        if (t_idle == 0) t_idle = now;
-                        else if (now - t_idle > kWaitLimitNs) {
-                            *abort_flag = 1;
-                            record_status(-7 /* ATTN_ERR_DEVICE_TIMEOUT */);
-                            ok = false;
-                        }
-                    }
+                    ok = pv(0, j);
                 }
+                if (ok) ok = pv(1, n_kv - 1);
             } else {
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j % C::kStages;
