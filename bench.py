@@ -56,6 +56,18 @@ WORKLOADS = {
     "paged": dict(kind="paged", Hq=32, Hkv=2, Sq=4096, D=256, NB=256, BS=512, L=100000,
                   scale=1.0 / 16, sets=1, seed0=1005,
                   name="paged_history_32q_2kv_d256_q4096_hist100000_fp8"),
+    # wider shapes the pages name beyond the five headline configurations
+    "vitl8k": dict(kind="encoder", B=1, H=16, S=8192, D=64, scale=0.125, sets=4, seed0=2100,
+                   name="vitl_native_b1_h16_s8192_d64"),
+    "enc_d128": dict(kind="encoder", B=1, H=16, S=2048, D=128, scale=128 ** -0.5, sets=12,
+                     seed0=2200, name="encoder_b1_h16_s2048_d128_x12"),
+    "gte": dict(kind="encoder", B=16, H=12, S=512, D=64, scale=0.125, sets=4, seed0=2300,
+                pad=(128, 512), name="gte_b16_h12_s512_d64_rightpad_128_512"),
+    "decode_d512": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=512, scale=512 ** -0.5,
+                        sets=4, seed0=2400, name="gqa_decode_b8_16q_8kv_d512_ctx4096"),
+    "decode_window": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=256, scale=1.0, sets=4,
+                          seed0=2500, window=1024,
+                          name="gqa_decode_b8_16q_8kv_d256_ctx4096_window1024"),
 }
 
 
@@ -159,10 +171,10 @@ class EncoderWork:
         self.sets = []
         self.host = []
         for i in range(cfg["sets"]):
-            c = syn.encoder_case(cfg["B"], cfg["H"], cfg["S"], cfg["D"], seed=cfg["seed0"] + i,
-                                 softmax_scale=cfg["scale"])
+            c = encoder_host_case(cfg, i)
             self.host.append(c)
             self.sets.append(tuple(t.to(device) for t in (c.q, c.k, c.v)))
+        self.bias = [c.key_bias.to(device) if c.key_bias is not None else None for c in self.host]
         self.out = [torch.empty_like(s[0]) for s in self.sets]
         B, H, S, D = cfg["B"], cfg["H"], cfg["S"], cfg["D"]
         self.flops_per_launch = 4.0 * B * H * S * S * D
@@ -175,8 +187,8 @@ class EncoderWork:
 
     def step(self, stream=None):
         from online_softmax_attention_flash_b200 import binding as Bd
-        for (q, k, v), o in zip(self.sets, self.out):
-            Bd.attn_encoder_fwd(q, k, v, self.cfg["scale"], out=o, stream=stream)
+        for (q, k, v), kb, o in zip(self.sets, self.bias, self.out):
+            Bd.attn_encoder_fwd(q, k, v, self.cfg["scale"], key_bias=kb, out=o, stream=stream)
 
     def rate(self, work, seconds):
         return work / seconds / 1e12
@@ -185,17 +197,22 @@ class EncoderWork:
     def e2e_setup(self):
         import torch
         self.h_in = [tuple(t.pin_memory() for t in (c.q, c.k, c.v)) for c in self.host]
+        self.h_bias = [c.key_bias.pin_memory() if c.key_bias is not None else None for c in self.host]
         self.h_out = [torch.empty_like(c.q).pin_memory() for c in self.host]
         self.h2d = sum(t.numel() * t.element_size() for s in self.h_in for t in s)
+        self.h2d += sum(t.numel() * t.element_size() for t in self.h_bias if t is not None)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
 
     def e2e_step(self, stream):
         from online_softmax_attention_flash_b200 import binding as Bd
-        for (hq, hk, hv), (q, k, v), o, ho in zip(self.h_in, self.sets, self.out, self.h_out):
+        for (hq, hk, hv), hb, (q, k, v), kb, o, ho in zip(self.h_in, self.h_bias, self.sets,
+                                                         self.bias, self.out, self.h_out):
+            if hb is not None:
+                kb.copy_(hb, non_blocking=True)
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
-            Bd.attn_encoder_fwd(q, k, v, self.cfg["scale"], out=o, stream=stream)
+            Bd.attn_encoder_fwd(q, k, v, self.cfg["scale"], key_bias=kb, out=o, stream=stream)
             ho.copy_(o, non_blocking=True)
 
     # CPU oracle on a bounded sample of the same workload
@@ -206,11 +223,44 @@ class EncoderWork:
         h = step_idx % self.cfg["H"]
         r0 = (step_idx * rows) % max(1, S - rows + 1) if S > rows else 0
         rr = np.arange(r0, min(S, r0 + rows))
-        q = c.q[0:1, h:h + 1].double().numpy()
-        k = c.k[0:1, h:h + 1].double().numpy()
-        v = c.v[0:1, h:h + 1].double().numpy()
-        oracle.encoder_attention(q, k, v, self.cfg["scale"], rows=rr)
+        b = step_idx % self.cfg["B"]
+        q = c.q[b:b + 1, h:h + 1].double().numpy()
+        k = c.k[b:b + 1, h:h + 1].double().numpy()
+        v = c.v[b:b + 1, h:h + 1].double().numpy()
+        kb = c.key_bias[b:b + 1].double().numpy() if c.key_bias is not None else None
+        oracle.encoder_attention(q, k, v, self.cfg["scale"], key_bias=kb, rows=rr)
         return 4.0 * len(rr) * S * self.cfg["D"], f"{len(rr)} query rows x {S} keys of one head"
+
+
+def encoder_host_case(cfg, i):
+    """Seeded encoder inputs; with cfg["pad"] = (lo, hi) every batch entry gets a right-padding
+    length drawn from U{lo..hi} (gte-style 0/1 attention mask as an additive key bias)."""
+    from online_softmax_attention_flash_b200 import inputs as syn
+    pads = None
+    if "pad" in cfg:
+        g = np.random.default_rng(cfg["seed0"] + 7919 * i)
+        pads = g.integers(cfg["pad"][0], cfg["pad"][1] + 1, size=cfg["B"]).tolist()
+    return syn.encoder_case(cfg["B"], cfg["H"], cfg["S"], cfg["D"], seed=cfg["seed0"] + i,
+                            softmax_scale=cfg["scale"], pad_lengths=pads)
+
+
+def decode_host_case(cfg, i):
+    """Seeded decode inputs; with cfg["window"] = W only the last W positions before each
+    length stay unmasked (sliding-window layers)."""
+    from online_softmax_attention_flash_b200 import inputs as syn
+    c = syn.decode_case(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"],
+                        seed=cfg["seed0"] + 100 * i, softmax_scale=cfg["scale"])
+    if "window" in cfg:
+        for b in range(cfg["B"]):
+            L = int(c.lengths[b])
+            c.attn_mask[b, ..., :max(0, L - cfg["window"])] = float("-inf")
+    return c
+
+
+def live_lengths(cfg, c):
+    """Keys each batch entry actually attends to (the bytes decode must read)."""
+    lens = [int(x) for x in c.lengths]
+    return [min(L, cfg["window"]) for L in lens] if "window" in cfg else lens
 
 
 class DecodeWork:
@@ -222,14 +272,13 @@ class DecodeWork:
         self.cfg = cfg
         self.host, self.sets = [], []
         for i in range(cfg["sets"]):
-            c = syn.decode_case(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"],
-                                seed=cfg["seed0"] + 100 * i, softmax_scale=cfg["scale"])
+            c = decode_host_case(cfg, i)
             self.host.append(c)
             self.sets.append(tuple(t.to(device) for t in (c.q, c.k, c.v, c.attn_mask)))
         self.out = [torch.empty_like(s[0]) for s in self.sets]
         ws = Bd.attn_gqa_decode_workspace_size(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"])
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
-        self.bytes = [oracle.decode_algorithmic_bytes(c.lengths.tolist(), cfg["Hkv"], cfg["D"],
+        self.bytes = [oracle.decode_algorithmic_bytes(live_lengths(cfg, c), cfg["Hkv"], cfg["D"],
                                                       cfg["Hq"], cfg["S"]) for c in self.host]
         self.launches_per_step = 3   # scan + stream + combine
         self.work_per_step = float(np.mean(self.bytes))
@@ -279,7 +328,7 @@ class DecodeWork:
                                     c.v[b:b + 1].double().numpy(),
                                     c.attn_mask[b:b + 1].double().numpy(), self.cfg["scale"],
                                     self.cfg["Hq"] // self.cfg["Hkv"])
-        L = int(c.lengths[b])
+        L = live_lengths(self.cfg, c)[b]
         byt = L * self.cfg["Hkv"] * self.cfg["D"] * 4 + 2 * self.cfg["Hq"] * self.cfg["D"] * 2
         return float(byt), "one batch entry (all heads) of the decode step"
 
@@ -347,7 +396,8 @@ class PagedWork:
 
 
 # steps captured per CUDA graph for the timed region (decode rotates 4 input sets)
-GRAPH_STEPS = {"vitl": 1, "tiny": 20, "dinov3": 20, "decode": 4, "paged": 1}
+GRAPH_STEPS = {"vitl": 1, "tiny": 20, "dinov3": 20, "decode": 4, "paged": 1, "vitl8k": 1,
+               "enc_d128": 1, "gte": 4, "decode_d512": 4, "decode_window": 4}
 
 
 def make_work(name, device):
@@ -411,13 +461,10 @@ def make_work_host_only(name):
     obj.cfg = cfg
     from online_softmax_attention_flash_b200 import inputs as syn
     if cfg["kind"] == "encoder":
-        obj.host = [syn.encoder_case(cfg["B"], cfg["H"], cfg["S"], cfg["D"], seed=cfg["seed0"] + i,
-                                     softmax_scale=cfg["scale"]) for i in range(cfg["sets"])]
+        obj.host = [encoder_host_case(cfg, i) for i in range(cfg["sets"])]
         obj.unit = "TFLOP/s"
     elif cfg["kind"] == "decode":
-        obj.host = [syn.decode_case(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["S"], cfg["D"],
-                                    seed=cfg["seed0"] + 100 * i, softmax_scale=cfg["scale"])
-                    for i in range(cfg["sets"])]
+        obj.host = [decode_host_case(cfg, i) for i in range(cfg["sets"])]
         obj.unit = "GB/s"
     else:
         obj.host = [syn.paged_case(cfg["Hq"], cfg["Hkv"], cfg["Sq"], cfg["D"], cfg["NB"], cfg["BS"],
@@ -571,7 +618,9 @@ def main(argv=None):
                    help="time eager calls instead of CUDA-graph replays")
     args = p.parse_args(argv)
     defaults = {"vitl": (1000, 20), "tiny": (2000, 20), "dinov3": (2000, 20),
-                "decode": (2000, 20), "paged": (100, 5)}[args.workload]
+                "decode": (2000, 20), "paged": (100, 5), "vitl8k": (400, 10),
+                "enc_d128": (1000, 20), "gte": (2000, 20), "decode_d512": (2000, 20),
+                "decode_window": (2000, 20)}[args.workload]
     if args.steps is None:
         args.steps = defaults[0]
     if args.warmup is None:

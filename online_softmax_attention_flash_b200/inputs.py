@@ -155,3 +155,13 @@ def gqa_decode_full_case() -> DecodeCase:
 def paged_full_case() -> PagedCase:
     return paged_case(32, 2, 4096, 256, num_phys_blocks=256, block_size=512,
                       actual_history_len=100000, seed=1005, softmax_scale=1.0 / 16.0)
+
+
+def rope_tables(S: int, D: int, base: float = 10000.0):
+    """cos / sin tables [S, D/2] fp32 for 1-D positions 0 .. S-1 with angle s * base^(-2j/D)
+    (pair j). The rotation kernels take any tables; models with 2-D or 3-D position grids
+    (DINOv3, V-JEPA2) only fill them differently."""
+    j = torch.arange(D // 2, dtype=torch.float64)
+    w = base ** (-2.0 * j / D)
+    theta = torch.arange(S, dtype=torch.float64)[:, None] * w[None, :]
+    return torch.cos(theta).float(), torch.sin(theta).float()

@@ -15,6 +15,7 @@ Modules
 attention   -- the definition for the three entry points (encoder, GQA decode,
                paged history) plus the split-KV log-sum-exp combine.
 e4m3        -- an FP8 E4M3FN decoder written from the format definition.
+rope        -- rotary position embedding of Q / K rows (both lane pairings).
 flops       -- the closed-form work counts used for throughput figures.
 """
 
@@ -27,4 +28,5 @@ from .attention import (  # noqa: F401
     lse_combine,
 )
 from .e4m3 import e4m3fn_to_float64  # noqa: F401
+from .rope import rope_apply, pair_lanes  # noqa: F401
 from .flops import attention_flops, decode_algorithmic_bytes  # noqa: F401
