@@ -68,6 +68,9 @@ WORKLOADS = {
     "decode_window": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=256, scale=1.0, sets=4,
                           seed0=2500, window=1024,
                           name="gqa_decode_b8_16q_8kv_d256_ctx4096_window1024"),
+    # the RoPE prologue of the ViT-L encoder (V-JEPA2 pairs lanes 2j, 2j+1), 24 layers
+    "rope_vitl": dict(kind="rope", B=1, H=16, S=2048, D=64, sets=24, seed0=2600, interleaved=True,
+                      name="rope_qk_vitl_b1_h16_s2048_d64_interleaved_x24layers"),
 }
 
 
@@ -333,6 +336,79 @@ class DecodeWork:
         return float(byt), "one batch entry (all heads) of the decode step"
 
 
+class RopeWork:
+    """attn_rope_qk over 24 distinct (q, k) sets; HBM bound: each call reads and writes q and k
+    and reads the [S, D/2] cos / sin tables."""
+
+    def __init__(self, cfg, device):
+        import torch
+        from online_softmax_attention_flash_b200 import inputs as syn
+        self.cfg = cfg
+        self.host = [rope_host_case(cfg, i) for i in range(cfg["sets"])]
+        self.sets = [tuple(t.to(device) for t in (q, k)) for q, k in self.host]
+        cos, sin = syn.rope_tables(cfg["S"], cfg["D"])
+        self.tables = (cos.to(device), sin.to(device))
+        self.h_tables = (cos, sin)
+        self.out = [(torch.empty_like(q), torch.empty_like(k)) for q, k in self.sets]
+        B, H, S, D = cfg["B"], cfg["H"], cfg["S"], cfg["D"]
+        self.bytes_per_call = 4.0 * B * H * S * D * 2 + 2.0 * S * (D // 2) * 4
+        self.launches_per_step = cfg["sets"]
+        self.work_per_step = self.bytes_per_call * cfg["sets"]
+        self.flops_per_launch = self.bytes_per_call
+        self.unit, self.bound = "GB/s", "hbm"
+        self.kernel_regex = "rope_qk_kernel"
+        self.peak_ratio = 1.0
+        self.dtype = "f32 (bf16 in / out)"
+
+    def step(self, stream=None):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        for (q, k), (qo, ko) in zip(self.sets, self.out):
+            Bd.attn_rope_qk(q, k, *self.tables, interleaved=self.cfg["interleaved"], q_out=qo,
+                            k_out=ko, stream=stream)
+
+    def rate(self, work, seconds):
+        return work / seconds / 1e9
+
+    def e2e_setup(self):
+        import torch
+        self.h_in = [tuple(t.pin_memory() for t in s) for s in self.host]
+        self.h_out = [tuple(torch.empty_like(t).pin_memory() for t in s) for s in self.host]
+        self.h2d = sum(t.numel() * t.element_size() for s in self.h_in for t in s)
+        self.d2h = sum(t.numel() * t.element_size() for s in self.h_out for t in s)
+
+    def e2e_step(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        for (hq, hk), (q, k), (qo, ko), (hqo, hko) in zip(self.h_in, self.sets, self.out, self.h_out):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            Bd.attn_rope_qk(q, k, *self.tables, interleaved=self.cfg["interleaved"], q_out=qo,
+                            k_out=ko, stream=stream)
+            hqo.copy_(qo, non_blocking=True)
+            hko.copy_(ko, non_blocking=True)
+
+    def e2e_work(self):
+        return self.work_per_step
+
+    def oracle_sample(self, step_idx):
+        import oracle
+        q, k = self.host[step_idx % len(self.host)]
+        h = step_idx % self.cfg["H"]
+        c, s = (t.double().numpy() for t in self.h_tables)
+        mode = "interleaved" if self.cfg["interleaved"] else "half"
+        for x in (q, k):
+            oracle.rope_apply(x[0, h].double().numpy(), c, s, mode)
+        S, D = self.cfg["S"], self.cfg["D"]
+        return 4.0 * S * D * 2 + 2.0 * S * (D // 2) * 4, "the q and k rows of one head"
+
+
+def rope_host_case(cfg, i):
+    from online_softmax_attention_flash_b200 import inputs as syn
+    import torch
+    g = torch.Generator().manual_seed(cfg["seed0"] + i)
+    shape = (cfg["B"], cfg["H"], cfg["S"], cfg["D"])
+    return syn.randn_bf16(shape, g), syn.randn_bf16(shape, g)
+
+
 class PagedWork:
     def __init__(self, cfg, device):
         import torch
@@ -397,12 +473,13 @@ class PagedWork:
 
 # steps captured per CUDA graph for the timed region (decode rotates 4 input sets)
 GRAPH_STEPS = {"vitl": 1, "tiny": 20, "dinov3": 20, "decode": 4, "paged": 1, "vitl8k": 1,
-               "enc_d128": 1, "gte": 4, "decode_d512": 4, "decode_window": 4}
+               "enc_d128": 1, "gte": 4, "decode_d512": 4, "decode_window": 4, "rope_vitl": 1}
 
 
 def make_work(name, device):
     cfg = WORKLOADS[name]
-    return {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork}[cfg["kind"]](cfg, device)
+    return {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork,
+            "rope": RopeWork}[cfg["kind"]](cfg, device)
 
 
 # --------------------------------------------------------------------- oracle
@@ -456,7 +533,8 @@ def run_reference(args, info):
 def make_work_host_only(name):
     """Host-side inputs only (the oracle arm never touches a GPU)."""
     cfg = WORKLOADS[name]
-    cls = {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork}[cfg["kind"]]
+    cls = {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork,
+           "rope": RopeWork}[cfg["kind"]]
     obj = cls.__new__(cls)
     obj.cfg = cfg
     from online_softmax_attention_flash_b200 import inputs as syn
@@ -465,6 +543,10 @@ def make_work_host_only(name):
         obj.unit = "TFLOP/s"
     elif cfg["kind"] == "decode":
         obj.host = [decode_host_case(cfg, i) for i in range(cfg["sets"])]
+        obj.unit = "GB/s"
+    elif cfg["kind"] == "rope":
+        obj.host = [rope_host_case(cfg, i) for i in range(cfg["sets"])]
+        obj.h_tables = syn.rope_tables(cfg["S"], cfg["D"])
         obj.unit = "GB/s"
     else:
         obj.host = [syn.paged_case(cfg["Hq"], cfg["Hkv"], cfg["Sq"], cfg["D"], cfg["NB"], cfg["BS"],
@@ -620,7 +702,7 @@ def main(argv=None):
     defaults = {"vitl": (1000, 20), "tiny": (2000, 20), "dinov3": (2000, 20),
                 "decode": (2000, 20), "paged": (100, 5), "vitl8k": (400, 10),
                 "enc_d128": (1000, 20), "gte": (2000, 20), "decode_d512": (2000, 20),
-                "decode_window": (2000, 20)}[args.workload]
+                "decode_window": (2000, 20), "rope_vitl": (1000, 20)}[args.workload]
     if args.steps is None:
         args.steps = defaults[0]
     if args.warmup is None:

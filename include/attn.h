@@ -193,6 +193,34 @@ ATTN_API int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const
                        uint16_t* out, void* stream);
 
 /*
+ * attn_rope_qk -- rotary position embedding of the query and key rows.
+ *
+ * Defined by: "vit-encoder-neuron-kernels", section "Kernels" (the encoder
+ * attention takes per-token rotation tables; two pairings of head-dim lanes).
+ * For every row (b, h, s) of q and of k and every pair j < D/2, with lanes
+ * (ia, ib) = (j, j + D/2) when interleaved == 0 ("half": DINOv3, EVA-02, Llama)
+ * or (2j, 2j + 1) when interleaved == 1 (V-JEPA2):
+ *     out[ia] = x[ia] cos[s][j] - x[ib] sin[s][j]
+ *     out[ib] = x[ia] sin[s][j] + x[ib] cos[s][j]
+ * computed in fp32 and rounded to bf16 (round-to-nearest-even). Apply it to Q and
+ * K before attn_encoder_fwd.
+ *
+ *   q, k          : [B, H, S, D] bf16 (device).
+ *   q_out, k_out  : [B, H, S, D] bf16 (device); may equal q / k (in place), must
+ *                   not otherwise overlap them or each other.
+ *   cos_table, sin_table : [S, D/2] fp32 (device), row s for token position s
+ *                   (any position grid: 1-D, or 2-D / 3-D patch grids flattened).
+ *   B, H, S >= 1; D a multiple of 16, 16 <= D <= 512.
+ * All pointers 16-byte aligned. Runs one kernel on `stream`; the caller owns all
+ * buffers.
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE (sizes, interleaved not 0 / 1, partial
+ * overlap), ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_ALIGN, ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_rope_qk(const uint16_t* q, const uint16_t* k, uint16_t* q_out, uint16_t* k_out,
+                          const float* cos_table, const float* sin_table,
+                          int B, int H, int S, int D, int interleaved, void* stream);
+
+/*
  * attn_check -- synchronise `stream`, then return and clear the first error the
  * device recorded on the current device since the last check (ATTN_OK if
  * none). Returns ATTN_ERR_CUDA if the synchronisation itself fails.

@@ -38,6 +38,7 @@ SIGNATURES = [
     ("attn_gqa_decode_noalloc", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     ("attn_paged_history", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _I, _I, _I, _I, _I,
                                 _P, _P]),
+    ("attn_rope_qk", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     ("attn_check", _I, [_P]),
     ("attn_status_string", ctypes.c_char_p, [_I]),
     ("attn_version", _I, []),
@@ -210,3 +211,23 @@ def attn_paged_history(q, k_cache, v_cache, block_table, block_size: int,
                                 int(num_kv_groups), Sq, D, _ptr(out), _stream_ptr(stream))
     _raise_if(st, "attn_paged_history")
     return out
+
+
+def attn_rope_qk(q, k, cos_table, sin_table, interleaved: bool = False, q_out=None, k_out=None,
+                 stream=None):
+    """Rotary embedding of q and k ([B, H, S, D] bf16) with cos / sin tables [S, D/2] fp32.
+    Returns (q_out, k_out); pass q_out=q, k_out=k to rotate in place."""
+    lib = load_library()
+    _need(q, "q", torch.bfloat16)
+    B, H, S, D = q.shape
+    _need(k, "k", torch.bfloat16, q.shape)
+    _need(cos_table, "cos_table", torch.float32, (S, D // 2))
+    _need(sin_table, "sin_table", torch.float32, (S, D // 2))
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    _need(q_out, "q_out", torch.bfloat16, q.shape)
+    _need(k_out, "k_out", torch.bfloat16, q.shape)
+    st = lib.attn_rope_qk(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _ptr(cos_table),
+                          _ptr(sin_table), B, H, S, D, 1 if interleaved else 0, _stream_ptr(stream))
+    _raise_if(st, "attn_rope_qk")
+    return q_out, k_out

@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "encoder.cuh"
 #include "paged.cuh"
+#include "rope.cuh"
 #include "tmap.cuh"
 
 namespace {
@@ -198,6 +199,29 @@ int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const uint8_t*
                                block_size, actual_history_len, k_scale, v_scale, softmax_scale,
                                Hq, Hkv, num_kv_groups, Sq, D, out,
                                static_cast<cudaStream_t>(stream));
+}
+
+int attn_rope_qk(const uint16_t* q, const uint16_t* k, uint16_t* q_out, uint16_t* k_out,
+                 const float* cos_table, const float* sin_table, int B, int H, int S, int D,
+                 int interleaved, void* stream) {
+    if (!q || !k || !q_out || !k_out || !cos_table || !sin_table) return ATTN_ERR_NULL;
+    if (B < 1 || H < 1 || S < 1 || D < 1 || (interleaved != 0 && interleaved != 1))
+        return ATTN_ERR_SHAPE;
+    if (D % 16 || D > 512) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out) ||
+        !aligned16(cos_table) || !aligned16(sin_table))
+        return ATTN_ERR_ALIGN;
+    // outputs may alias their own input exactly; any other overlap is rejected
+    const size_t bytes = static_cast<size_t>(B) * H * S * D * 2;
+    auto overlap = [bytes](const void* a, const void* b) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+        return x < y + bytes && y < x + bytes;
+    };
+    if ((q_out != q && overlap(q_out, q)) || (k_out != k && overlap(k_out, k)) ||
+        overlap(q_out, k_out) || overlap(q_out, k) || overlap(k_out, q))
+        return ATTN_ERR_SHAPE;
+    return attn::rope::launch(q, k, q_out, k_out, cos_table, sin_table, B, H, S, D,
+                              interleaved != 0, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -101,3 +101,17 @@ def test_noalloc_size_limit_is_checked_on_the_host(lib):
                                        1.0, None) == -5
     assert lib.attn_gqa_decode_noalloc(fake, fake, fake, None, fake, 0, 16, 8, 2, 64, 256,
                                        1.0, None) == -2
+
+
+def test_rope_validation_rejects_before_any_launch(lib):
+    fake = [ctypes.c_void_p(4096 * (i + 1) * 1024 * 1024) for i in range(6)]   # never dereferenced
+    q, k, qo, ko, c, s = fake
+    f = lib.attn_rope_qk
+    assert f(None, k, qo, ko, c, s, 1, 1, 8, 64, 0, None) == -1                 # NULL
+    assert f(q, k, qo, ko, c, s, 0, 1, 8, 64, 0, None) == -2                    # B < 1
+    assert f(q, k, qo, ko, c, s, 1, 1, 8, 64, 2, None) == -2                    # pairing flag
+    assert f(q, k, qo, ko, c, s, 1, 1, 8, 72, 0, None) == -3                    # D % 16
+    assert f(q, k, qo, ko, c, s, 1, 1, 8, 1024, 0, None) == -3                  # D > 512
+    assert f(ctypes.c_void_p(4096 + 8), k, qo, ko, c, s, 1, 1, 8, 64, 0, None) == -4
+    assert f(q, k, ctypes.c_void_p(q.value + 256), ko, c, s, 1, 1, 8, 64, 0, None) == -2  # overlap
+    assert f(q, k, ko, ko, c, s, 1, 1, 8, 64, 0, None) == -2                    # q_out == k_out
