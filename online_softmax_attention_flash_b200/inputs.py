@@ -132,6 +132,49 @@ def paged_case(Hq, Hkv, Sq, D, num_phys_blocks, block_size, actual_history_len, 
                      Hq // Hkv)
 
 
+@dataclass
+class PagedPrefillCase:
+    q: torch.Tensor            # [Hq, total_q, D] bf16, the sequences' current tokens packed
+    k_cache: torch.Tensor      # [num_phys_blocks, Hkv, block_size, D] uint8 (E4M3FN codes)
+    v_cache: torch.Tensor
+    k_scale: float
+    v_scale: float
+    block_tables: torch.Tensor  # [num_seqs, max_blocks] int32 (-1 past each sequence's blocks)
+    block_size: int
+    q_start: torch.Tensor      # [num_seqs + 1] int32, row offsets into q
+    hist_lens: torch.Tensor    # [num_seqs] int32
+    softmax_scale: float
+    num_kv_groups: int
+
+
+def paged_prefill_case(Hq, Hkv, D, block_size, hist_lens, q_lens, seed, softmax_scale=None,
+                       spare_blocks=3) -> PagedPrefillCase:
+    """Sequences with the given history and current lengths; each owns a disjoint random set
+    of physical blocks covering hist + q_len positions (current tokens' K/V included)."""
+    g = _gen(seed)
+    need = [-(-(int(h) + int(n)) // block_size) for h, n in zip(hist_lens, q_lens)]
+    nb = sum(need) + spare_blocks
+    kf = torch.randn((nb, Hkv, block_size, D), generator=g, dtype=torch.float32)
+    vf = torch.randn((nb, Hkv, block_size, D), generator=g, dtype=torch.float32)
+    kc, ks = quantize_e4m3fn(kf)
+    vc, vs = quantize_e4m3fn(vf)
+    perm = torch.randperm(nb, generator=g).to(torch.int32)
+    tables = torch.full((len(need), max(need + [1])), -1, dtype=torch.int32)
+    o = 0
+    for s, n in enumerate(need):
+        tables[s, :n] = perm[o:o + n]
+        o += n
+    starts = [0]
+    for n in q_lens:
+        starts.append(starts[-1] + int(n))
+    q = randn_bf16((Hq, starts[-1], D), g)
+    scale = (1.0 / D ** 0.5) if softmax_scale is None else float(softmax_scale)
+    return PagedPrefillCase(q, kc, vc, ks, vs, tables.contiguous(), block_size,
+                            torch.tensor(starts, dtype=torch.int32),
+                            torch.tensor([int(h) for h in hist_lens], dtype=torch.int32), scale,
+                            Hq // Hkv)
+
+
 # The five workloads named by the pages' shapes.
 def tiny_case() -> EncoderCase:
     return encoder_case(1, 4, 256, 64, seed=1001, softmax_scale=0.125)

@@ -12,8 +12,9 @@ in float64, two passes per query row (row max, then exp / sum / P V).
 
 Modules
 -------
-attention   -- the definition for the three entry points (encoder, GQA decode,
-               paged history) plus the split-KV log-sum-exp combine.
+attention   -- the definition for the entry points (encoder, GQA decode, paged
+               history, paged prefill with causal current tokens) plus the
+               split-KV log-sum-exp combine.
 e4m3        -- an FP8 E4M3FN decoder written from the format definition.
 rope        -- rotary position embedding of Q / K rows (both lane pairings).
 flops       -- the closed-form work counts used for throughput figures.
@@ -24,6 +25,7 @@ from .attention import (  # noqa: F401
     encoder_attention,
     gqa_decode_attention,
     paged_history_attention,
+    paged_prefill_attention,
     paged_logical_kv,
     lse_combine,
 )

@@ -164,6 +164,41 @@ def paged_history_attention(q, k_codes, v_codes, k_scale, v_scale, block_table, 
     return out[0]
 
 
+def paged_prefill_attention(q, k_codes, v_codes, k_scale, v_scale, block_tables, block_size,
+                            q_start, hist_lens, softmax_scale, num_kv_groups, rows=None):
+    """Prefill attention over a paged FP8 cache: history plus the current tokens, causal
+    among the current tokens (the PCP history page's "current tokens do not attend to one
+    another yet", completed; several sequences per call).
+
+    q [Hq, total_q, D]: the current tokens of num_seqs sequences, packed; sequence s owns
+    rows q_start[s] .. q_start[s+1] - 1. Its K/V, history and current tokens alike, sit in
+    the cache at logical positions 0 .. hist_lens[s] + q_len_s - 1 of block_tables[s].
+    Query i of sequence s is at logical position hist_lens[s] + i and attends to every
+    position t <= hist_lens[s] + i. ``rows`` optionally restricts the evaluated rows of
+    each sequence (indices into 0 .. q_len_s - 1, those past q_len_s are skipped); the
+    result keeps the [Hq, total_q, D] layout with unevaluated rows left 0.
+    """
+    q = _as_f64(q)
+    Hq, total_q, D = q.shape
+    out = np.zeros_like(q)
+    starts = [int(x) for x in q_start]
+    for s, hist in enumerate(int(x) for x in hist_lens):
+        a, b = starts[s], starts[s + 1]
+        n = b - a
+        if n == 0:
+            continue
+        kl, vl = paged_logical_kv(k_codes, v_codes, k_scale, v_scale, block_tables[s],
+                                  block_size, hist + n)
+        i = np.arange(n)[:, None]
+        t = np.arange(hist + n)[None, :]
+        mask = np.where(t <= hist + i, 0.0, -np.inf)[None, None]
+        r = np.arange(n) if rows is None else np.asarray([x for x in rows if x < n], dtype=np.int64)
+        o = softmax_attention(q[None, :, a:b], kl[None], vl[None], softmax_scale, num_kv_groups,
+                              mask, rows=r)
+        out[:, a + r] = o[0]
+    return out
+
+
 def lse_combine(o_parts, m_parts, l_parts):
     """Combine split-KV partial results of one query row.
 
