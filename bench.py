@@ -68,6 +68,10 @@ WORKLOADS = {
     "decode_window": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=256, scale=1.0, sets=4,
                           seed0=2500, window=1024,
                           name="gqa_decode_b8_16q_8kv_d256_ctx4096_window1024"),
+    # chunked prefill over the paged FP8 cache: 8 sequences, history + causal current tokens
+    "paged_prefill": dict(kind="prefill", Hq=32, Hkv=2, D=256, BS=512, n_seqs=8,
+                          hist=(4096, 16384), qlen=(512, 2048), scale=1.0 / 16, sets=1,
+                          seed0=2700, name="paged_prefill_8seq_32q_2kv_d256_hist4k_16k_q512_2k_fp8"),
     # the RoPE prologue of the ViT-L encoder (V-JEPA2 pairs lanes 2j, 2j+1), 24 layers
     "rope_vitl": dict(kind="rope", B=1, H=16, S=2048, D=64, sets=24, seed0=2600, interleaved=True,
                       name="rope_qk_vitl_b1_h16_s2048_d64_interleaved_x24layers"),
@@ -471,15 +475,91 @@ class PagedWork:
         return 4.0 * len(rr) * self.cfg["L"] * self.cfg["D"], f"{len(rr)} query rows of one head"
 
 
+def prefill_host_case(cfg):
+    from online_softmax_attention_flash_b200 import inputs as syn
+    g = np.random.default_rng(cfg["seed0"])
+    hist = g.integers(cfg["hist"][0], cfg["hist"][1] + 1, size=cfg["n_seqs"]).tolist()
+    qlen = g.integers(cfg["qlen"][0], cfg["qlen"][1] + 1, size=cfg["n_seqs"]).tolist()
+    return syn.paged_prefill_case(cfg["Hq"], cfg["Hkv"], cfg["D"], cfg["BS"], hist, qlen,
+                                  seed=cfg["seed0"], softmax_scale=cfg["scale"])
+
+
+def prefill_flops(c, Hq, D):
+    """4 * Hq * D per (query, visible key) pair: query i of a sequence sees hist + i + 1 keys."""
+    tot = 0
+    for s in range(len(c.hist_lens)):
+        n = int(c.q_start[s + 1] - c.q_start[s])
+        h = int(c.hist_lens[s])
+        tot += n * h + n * (n + 1) // 2
+    return 4.0 * Hq * D * tot
+
+
+class PrefillWork(PagedWork):
+    """attn_paged_prefill on several sequences (fp8 MMAs, like the history kernel)."""
+
+    def __init__(self, cfg, device):
+        import torch
+        self.cfg = cfg
+        c = prefill_host_case(cfg)
+        self.host = [c]
+        self.dev = tuple(t.to(device) for t in (c.q, c.k_cache, c.v_cache, c.block_tables,
+                                                c.q_start, c.hist_lens))
+        self.max_q = int((c.q_start[1:] - c.q_start[:-1]).max())
+        self.out = torch.empty_like(self.dev[0])
+        self.flops_per_launch = prefill_flops(c, cfg["Hq"], cfg["D"])
+        self.launches_per_step = 1
+        self.work_per_step = self.flops_per_launch
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.kernel_regex = "paged_history_kernel"
+        self.peak_ratio = 2.0
+        self.dtype = "e4m3 (q and p as hi+lo e4m3 pairs), fp32 accumulate"
+
+    def _call(self, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        c = self.host[0]
+        q, kc, vc, bt, qs, hl = self.dev
+        Bd.attn_paged_prefill(q, kc, vc, bt, qs, hl, c.k_scale, c.v_scale, c.softmax_scale,
+                              c.num_kv_groups, max_q_len=self.max_q, out=self.out, stream=stream)
+
+    def e2e_setup(self):
+        import torch
+        c = self.host[0]
+        self.h_in = tuple(t.pin_memory() for t in (c.q, c.k_cache, c.v_cache, c.block_tables,
+                                                   c.q_start, c.hist_lens))
+        self.h_out = torch.empty_like(c.q).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def oracle_sample(self, step_idx, rows=16):
+        import oracle
+        import torch
+        c = self.host[0]
+        s = step_idx % len(c.hist_lens)
+        h = step_idx % self.cfg["Hq"]
+        g = h // c.num_kv_groups
+        a, b = int(c.q_start[s]), int(c.q_start[s + 1])
+        r0 = (step_idx * rows) % (b - a)
+        rr = np.arange(r0, min(b - a, r0 + rows))
+        oracle.paged_prefill_attention(c.q[h:h + 1, a:b].double().numpy(), c.k_cache[:, g:g + 1].numpy(),
+                                       c.v_cache[:, g:g + 1].numpy(), c.k_scale, c.v_scale,
+                                       c.block_tables[s:s + 1].numpy(), c.block_size,
+                                       np.array([0, b - a]), c.hist_lens[s:s + 1].numpy(),
+                                       c.softmax_scale, 1, rows=rr)
+        hist = int(c.hist_lens[s])
+        pairs = sum(hist + int(i) + 1 for i in rr)
+        return 4.0 * pairs * self.cfg["D"], f"{len(rr)} query rows of one head of one sequence"
+
+
 # steps captured per CUDA graph for the timed region (decode rotates 4 input sets)
 GRAPH_STEPS = {"vitl": 1, "tiny": 20, "dinov3": 20, "decode": 4, "paged": 1, "vitl8k": 1,
-               "enc_d128": 1, "gte": 4, "decode_d512": 4, "decode_window": 4, "rope_vitl": 1}
+               "enc_d128": 1, "gte": 4, "decode_d512": 4, "decode_window": 4, "rope_vitl": 1,
+               "paged_prefill": 1}
 
 
 def make_work(name, device):
     cfg = WORKLOADS[name]
     return {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork,
-            "rope": RopeWork}[cfg["kind"]](cfg, device)
+            "rope": RopeWork, "prefill": PrefillWork}[cfg["kind"]](cfg, device)
 
 
 # --------------------------------------------------------------------- oracle
@@ -534,7 +614,7 @@ def make_work_host_only(name):
     """Host-side inputs only (the oracle arm never touches a GPU)."""
     cfg = WORKLOADS[name]
     cls = {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork,
-           "rope": RopeWork}[cfg["kind"]]
+           "rope": RopeWork, "prefill": PrefillWork}[cfg["kind"]]
     obj = cls.__new__(cls)
     obj.cfg = cfg
     from online_softmax_attention_flash_b200 import inputs as syn
@@ -544,6 +624,9 @@ def make_work_host_only(name):
     elif cfg["kind"] == "decode":
         obj.host = [decode_host_case(cfg, i) for i in range(cfg["sets"])]
         obj.unit = "GB/s"
+    elif cfg["kind"] == "prefill":
+        obj.host = [prefill_host_case(cfg)]
+        obj.unit = "TFLOP/s"
     elif cfg["kind"] == "rope":
         obj.host = [rope_host_case(cfg, i) for i in range(cfg["sets"])]
         obj.h_tables = syn.rope_tables(cfg["S"], cfg["D"])
@@ -670,7 +753,7 @@ def run_product(args, info):
         "config": {"workload": cfg["name"],
                    **{k: v for k, v in cfg.items() if k not in ("kind", "name", "seed0")},
                    "l2": ("inputs larger than L2: distinct input sets rotate across calls"
-                          if cfg["sets"] > 1 or cfg["kind"] == "paged" else "inputs fit in L2"),
+                          if cfg["sets"] > 1 or cfg["kind"] in ("paged", "prefill") else "inputs fit in L2"),
                    "parallelism": f"replicas x{info.world_size}", "launch": launch_mode},
         "step_ms": {"min": s_sorted[0], "median": statistics.median(step_ms),
                     "mean": statistics.fmean(step_ms),
@@ -702,7 +785,8 @@ def main(argv=None):
     defaults = {"vitl": (1000, 20), "tiny": (2000, 20), "dinov3": (2000, 20),
                 "decode": (2000, 20), "paged": (100, 5), "vitl8k": (400, 10),
                 "enc_d128": (1000, 20), "gte": (2000, 20), "decode_d512": (2000, 20),
-                "decode_window": (2000, 20), "rope_vitl": (1000, 20)}[args.workload]
+                "decode_window": (2000, 20), "rope_vitl": (1000, 20),
+                "paged_prefill": (30, 5)}[args.workload]
     if args.steps is None:
         args.steps = defaults[0]
     if args.warmup is None:

@@ -53,7 +53,8 @@ typedef enum attn_status {
     ATTN_ERR_WORKSPACE = -5,      /* workspace missing or too small                  */
     ATTN_ERR_CUDA = -6,           /* a CUDA runtime / driver call failed             */
     ATTN_ERR_DEVICE_TIMEOUT = -7, /* a kernel's bounded wait ran out (device side)   */
-    ATTN_ERR_BLOCK_TABLE = -8     /* a block-table entry is outside the pool (device)*/
+    ATTN_ERR_BLOCK_TABLE = -8,    /* a block-table entry is outside the pool (device)*/
+    ATTN_ERR_SEQUENCE = -9        /* a sequence descriptor is out of range (device)  */
 } attn_status;
 
 /*
@@ -182,6 +183,9 @@ ATTN_API int attn_gqa_decode_noalloc(const uint16_t* q, const uint16_t* k, const
  *   Every query attends to every history position < len (no causal mask).
  * Table entries are checked on the device: an entry outside
  * [0, num_phys_blocks) is skipped and recorded as ATTN_ERR_BLOCK_TABLE.
+ * Cache rows past len inside the last block read are multiplied by a zero
+ * probability, so they must hold finite codes (any value; E4M3FN quantisation
+ * never writes the two NaN codes).
  * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_ALIGN,
  * ATTN_ERR_CUDA.
  */
@@ -191,6 +195,48 @@ ATTN_API int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const
                        float k_scale, float v_scale, float softmax_scale,
                        int Hq, int Hkv, int num_kv_groups, int Sq, int D,
                        uint16_t* out, void* stream);
+
+/*
+ * attn_paged_prefill -- prefill attention over a paged FP8 KV cache: each
+ * sequence's current tokens attend to its history and, causally, to each other.
+ *
+ * Defined by: "Prefill Context-Parallel Attention POC for Trainium2" (layout and
+ * constraints as attn_paged_history), completing its "current tokens do not
+ * attend to one another yet": the current tokens' K/V are written into the cache
+ * after the history first (as E4M3FN codes, like the history), then
+ *     out[h, q0 + i] = softmax_t(scale * q[h, q0 + i] . K_t) V_t,
+ *     t over logical positions 0 .. hist + i of the sequence's block table,
+ * for query i of a sequence whose rows start at q0 and whose history has hist
+ * tokens. Several sequences per call.
+ *
+ *   q           : [Hq, total_q, D] bf16, the sequences' current tokens packed
+ *   k_cache, v_cache : [num_phys_blocks, Hkv, block_size, D] E4M3FN codes
+ *   block_tables: [num_seqs, table_stride] int32 (device); row s maps sequence
+ *                 s's logical blocks to physical blocks
+ *   q_start     : [num_seqs + 1] int32 (device), non-decreasing row offsets,
+ *                 q_start[0] = 0, q_start[num_seqs] = total_q
+ *   hist_lens   : [num_seqs] int32 (device), >= 0, with hist + q_len <=
+ *                 table_stride * block_size
+ *   max_q_len   : host bound on every q_len (sizes the grid)
+ *   k_scale, v_scale, softmax_scale, Hq, Hkv, num_kv_groups, D, block_size:
+ *                 as attn_paged_history (D == 256)
+ *   out         : [Hq, total_q, D] bf16
+ * Cache rows past a sequence's last position inside its last block must hold
+ * finite codes, as for attn_paged_history.
+ * num_seqs <= 65535. The device checks every sequence descriptor (a bad one
+ * writes nothing for that sequence and records ATTN_ERR_SEQUENCE) and every
+ * table entry it reads (ATTN_ERR_BLOCK_TABLE). Only blocks up to each tile's
+ * last visible position are read.
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_ALIGN,
+ * ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_paged_prefill(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                                const int32_t* block_tables, int table_stride, int num_phys_blocks,
+                                int block_size, const int32_t* q_start, const int32_t* hist_lens,
+                                int num_seqs, int total_q, int max_q_len,
+                                float k_scale, float v_scale, float softmax_scale,
+                                int Hq, int Hkv, int num_kv_groups, int D,
+                                uint16_t* out, void* stream);
 
 /*
  * attn_rope_qk -- rotary position embedding of the query and key rows.

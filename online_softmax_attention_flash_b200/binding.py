@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_PKG_DIR, "libattn_b200.so")
 STATUS = {
     0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_UNSUPPORTED",
     -4: "ATTN_ERR_ALIGN", -5: "ATTN_ERR_WORKSPACE", -6: "ATTN_ERR_CUDA",
-    -7: "ATTN_ERR_DEVICE_TIMEOUT", -8: "ATTN_ERR_BLOCK_TABLE",
+    -7: "ATTN_ERR_DEVICE_TIMEOUT", -8: "ATTN_ERR_BLOCK_TABLE", -9: "ATTN_ERR_SEQUENCE",
 }
 
 # (name, restype, argtypes) for every symbol declared in include/attn.h
@@ -38,6 +38,8 @@ SIGNATURES = [
     ("attn_gqa_decode_noalloc", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     ("attn_paged_history", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _I, _I, _I, _I, _I,
                                 _P, _P]),
+    ("attn_paged_prefill", _I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _F, _F, _F, _I, _I,
+                                _I, _I, _P, _P]),
     ("attn_rope_qk", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     ("attn_check", _I, [_P]),
     ("attn_status_string", ctypes.c_char_p, [_I]),
@@ -210,6 +212,42 @@ def attn_paged_history(q, k_cache, v_cache, block_table, block_size: int,
                                 float(k_scale), float(v_scale), float(softmax_scale), Hq, Hkv,
                                 int(num_kv_groups), Sq, D, _ptr(out), _stream_ptr(stream))
     _raise_if(st, "attn_paged_history")
+    return out
+
+
+def attn_paged_prefill(q, k_cache, v_cache, block_tables, q_start, hist_lens, k_scale: float,
+                       v_scale: float, softmax_scale: float, num_kv_groups: int, max_q_len=None,
+                       out=None, stream=None):
+    """q [Hq, total_q, D] bf16 (current tokens of all sequences, packed); k/v_cache
+    [NB, Hkv, block_size, D] uint8 codes holding history AND current tokens; block_tables
+    [num_seqs, stride] int32; q_start [num_seqs + 1] int32; hist_lens [num_seqs] int32 (all
+    CUDA). max_q_len: host bound on the sequences' current lengths (read from q_start on the
+    host if None). Returns out [Hq, total_q, D] bf16."""
+    lib = load_library()
+    _need(q, "q", torch.bfloat16)
+    Hq, total_q, D = q.shape
+    _need(k_cache, "k_cache", torch.uint8)
+    NB, Hkv, BS, Dk = k_cache.shape
+    if Dk != D:
+        raise ValueError("k_cache must be [num_phys_blocks, Hkv, block_size, D]")
+    _need(v_cache, "v_cache", torch.uint8, k_cache.shape)
+    _need(block_tables, "block_tables", torch.int32)
+    if block_tables.dim() != 2:
+        raise ValueError("block_tables must be [num_seqs, stride]")
+    num_seqs, stride = block_tables.shape
+    _need(q_start, "q_start", torch.int32, (num_seqs + 1,))
+    _need(hist_lens, "hist_lens", torch.int32, (num_seqs,))
+    if max_q_len is None:
+        qs = q_start.cpu()
+        max_q_len = int((qs[1:] - qs[:-1]).max()) if num_seqs > 0 else 0
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, q.shape)
+    st = lib.attn_paged_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), stride, NB,
+                                BS, _ptr(q_start), _ptr(hist_lens), num_seqs, total_q, int(max_q_len),
+                                float(k_scale), float(v_scale), float(softmax_scale), Hq, Hkv,
+                                int(num_kv_groups), D, _ptr(out), _stream_ptr(stream))
+    _raise_if(st, "attn_paged_prefill")
     return out
 
 

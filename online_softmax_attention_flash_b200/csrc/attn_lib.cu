@@ -103,6 +103,7 @@ const char* attn_status_string(int status) {
         case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
         case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT";
         case ATTN_ERR_BLOCK_TABLE: return "ATTN_ERR_BLOCK_TABLE";
+        case ATTN_ERR_SEQUENCE: return "ATTN_ERR_SEQUENCE";
         default: return "ATTN_ERR_UNKNOWN";
     }
 }
@@ -199,6 +200,32 @@ int attn_paged_history(const uint16_t* q, const uint8_t* k_cache, const uint8_t*
                                block_size, actual_history_len, k_scale, v_scale, softmax_scale,
                                Hq, Hkv, num_kv_groups, Sq, D, out,
                                static_cast<cudaStream_t>(stream));
+}
+
+int attn_paged_prefill(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                       const int32_t* block_tables, int table_stride, int num_phys_blocks,
+                       int block_size, const int32_t* q_start, const int32_t* hist_lens,
+                       int num_seqs, int total_q, int max_q_len, float k_scale, float v_scale,
+                       float softmax_scale, int Hq, int Hkv, int num_kv_groups, int D,
+                       uint16_t* out, void* stream) {
+    if (!q || !k_cache || !v_cache || !block_tables || !q_start || !hist_lens || !out)
+        return ATTN_ERR_NULL;
+    if (Hq < 1 || Hkv < 1 || num_kv_groups < 1 || Hq != Hkv * num_kv_groups) return ATTN_ERR_SHAPE;
+    if (num_seqs < 1 || num_seqs > 65535 || total_q < 0 || max_q_len < 0 || table_stride < 1 ||
+        num_phys_blocks < 1)
+        return ATTN_ERR_SHAPE;
+    if (block_size < 128 || block_size > 512 || block_size % 128) return ATTN_ERR_SHAPE;
+    if (!scale_ok(softmax_scale) || !scale_ok(k_scale) || !std::isfinite(v_scale)) return ATTN_ERR_SHAPE;
+    if (D != 256) return ATTN_ERR_UNSUPPORTED;
+    if (Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(q_start) & 3u) ||
+        (reinterpret_cast<uintptr_t>(hist_lens) & 3u))
+        return ATTN_ERR_ALIGN;
+    return attn::paged::launch_prefill(q, k_cache, v_cache, block_tables, table_stride,
+                                       num_phys_blocks, block_size, q_start, hist_lens, num_seqs,
+                                       total_q, max_q_len, k_scale, v_scale, softmax_scale, Hq, Hkv,
+                                       num_kv_groups, out, static_cast<cudaStream_t>(stream));
 }
 
 int attn_rope_qk(const uint16_t* q, const uint16_t* k, uint16_t* q_out, uint16_t* k_out,

@@ -25,6 +25,14 @@
 //   * S is double-buffered in TMEM so QK of the next sub-tile runs while the
 //     softmax warpgroup works; P_hi / P_lo are written back over S and read by
 //     the MMA from TMEM; O (128 x 256 fp32) stays in TMEM for the whole loop.
+//
+// Prefill with current tokens (the same kernel, `Params::seq_q_start` set): the page's
+// "current tokens do not attend to one another yet", completed. Several sequences per
+// launch (blockIdx.z); sequence s owns q rows seq_q_start[s] .. seq_q_start[s+1] - 1,
+// its block-table row and history length seq_hist[s]; its current tokens' K/V are in
+// the cache after the history. Query i (logical position hist + i) sees every position
+// t <= hist + i: each softmax row masks its own limit, and a CTA loads only the
+// sub-tiles its last row can see.
 #pragma once
 
 #include "ptx.cuh"
@@ -84,18 +92,22 @@ __device__ __forceinline__ Bars carve(uint8_t* smem) {
 
 struct Params {
     uint16_t* out;
-    const int32_t* block_table;
-    int Sq, Hkv, G, num_phys_blocks, block_size, hist_len, n_sub;
+    const int32_t* block_table;     // history mode: the table; prefill: row 0 of [num_seqs][table_stride]
+    int Sq, Hkv, G, num_phys_blocks, block_size, hist_len;
     float c_qk;        // k_scale * softmax_scale * log2(e)   (times the per-row Q scale)
     float v_scale;
+    // prefill with current tokens (nullptr: one sequence, history only)
+    const int32_t* seq_q_start;     // [num_seqs + 1]
+    const int32_t* seq_hist;        // [num_seqs]
+    int table_stride;               // block-table entries per sequence
 };
 
 // Logical 128-key sub-tile j -> (physical block, row offset); -1 if the table entry is bad.
-__device__ __forceinline__ int sub_tile_block(const Params& p, int j, int* off) {
+__device__ __forceinline__ int sub_tile_block(const Params& p, const int32_t* table, int j, int* off) {
     const int t0 = j * kTileN;
     const int lb = t0 / p.block_size;
     *off = t0 - lb * p.block_size;
-    const int phys = __ldg(p.block_table + lb);
+    const int phys = __ldg(table + lb);
     return (phys >= 0 && phys < p.num_phys_blocks) ? phys : -1;
 }
 
@@ -111,8 +123,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int warp = threadIdx.x >> 5;
     const int h = blockIdx.y;
     const int g = h / p.G;
-    const int row0 = blockIdx.x * kTileM;
-    const int n_sub = p.n_sub;
+    const int row0 = blockIdx.x * kTileM;   // first query row of the tile, within its sequence
 
     if (threadIdx.x == 0) {
         mbar_init(bars.q_full, 1);
@@ -142,7 +153,32 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     pdl_launch_dependents();
     pdl_wait_predecessor();
 
-    if (warp == kProducerWarp) {
+    // this CTA's sequence: q rows [q0, q0 + q_len), history length, block-table row
+    int q0 = 0, q_len = p.Sq, hist = p.hist_len;
+    const int32_t* table = p.block_table;
+    const bool causal = p.seq_q_start != nullptr;
+    bool active = true;
+    if (causal) {
+        const int s = blockIdx.z;
+        q0 = __ldg(p.seq_q_start + s);
+        q_len = __ldg(p.seq_q_start + s + 1) - q0;
+        hist = __ldg(p.seq_hist + s);
+        table = p.block_table + static_cast<size_t>(s) * p.table_stride;
+        if (q0 < 0 || q_len < 0 || q0 + q_len > p.Sq || hist < 0 ||
+            static_cast<long long>(hist) + q_len > static_cast<long long>(p.table_stride) * p.block_size) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+                record_status(-9 /* ATTN_ERR_SEQUENCE */);
+            active = false;
+        }
+    }
+    active = active && row0 < q_len;
+    // keys [0, key_end) are visible to some row of the tile
+    const int key_end = causal ? hist + min(row0 + kTileM, q_len) : hist;
+    const int n_sub = active ? (key_end + kTileN - 1) / kTileN : 0;
+
+    if (!active) {
+        // nothing to compute or store (rows past the sequence, or a bad descriptor)
+    } else if (warp == kProducerWarp) {
         // ---------------------------------------------------------------- producer
         if (lane_id() == 0) {
             prefetch_tensormap(&tm_q);
@@ -150,7 +186,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             prefetch_tensormap(&tm_v);
             mbar_arrive_expect_tx(bars.q_full, 4 * kPanel);
             for (int pn = 0; pn < 4; ++pn)
-                tma_load_3d(smem + kStageOff + pn * kPanel, &tm_q, bars.q_full, pn * 64, row0, h);
+                tma_load_3d(smem + kStageOff + pn * kPanel, &tm_q, bars.q_full, pn * 64, q0 + row0, h);
             // the ring doubles as Q staging until the softmax warps have quantised Q
             bool ok = mbar_wait(bars.q_ready, 0, abort_flag);
             int issued = 0;
@@ -158,7 +194,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int st = j % kStages;
                 const uint32_t use = j / kStages;
                 int off;
-                int phys = sub_tile_block(p, j, &off);
+                int phys = sub_tile_block(p, table, j, &off);
                 if (phys < 0) {
                     record_status(-8 /* ATTN_ERR_BLOCK_TABLE */);
                     phys = 0;   // load something valid; the softmax masks the whole sub-tile
@@ -328,8 +364,10 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int b = j & 1;
             const uint32_t tS = tmem_base + lane_off + kColS0 + b * 128;
             int off;
-            const bool blk_ok = sub_tile_block(p, j, &off) >= 0;
-            const int valid = blk_ok ? min(kTileN, p.hist_len - j * kTileN) : 0;
+            const bool blk_ok = sub_tile_block(p, table, j, &off) >= 0;
+            // this row sees keys [0, lim): the history, plus current tokens up to itself
+            const int lim = causal ? hist + row0 + r + 1 : hist;
+            const int valid = blk_ok ? max(0, min(kTileN, lim - j * kTileN)) : 0;
             ok = mbar_wait(&bars.s_full[b], (j >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
@@ -407,7 +445,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (ok) {
             tc_fence_after();
             const int row = row0 + r;
-            uint16_t* orow = p.out + (static_cast<size_t>(h) * p.Sq + row) * kD;
+            uint16_t* orow = p.out + (static_cast<size_t>(h) * p.Sq + q0 + row) * kD;
             const bool live = l_run > 0.f;
             const float f = live ? p.v_scale / l_run : 0.f;
 #pragma unroll
@@ -419,7 +457,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 for (int i = 0; i < 16; ++i)
                     pk[i] = live ? pack_bf16x2(__uint_as_float(u[2 * i]) * f, __uint_as_float(u[2 * i + 1]) * f)
                                  : 0u;
-                if (row < p.Sq) {
+                if (row < q_len) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
@@ -437,12 +475,10 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
 }
 
-inline int launch(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
-                  const int32_t* block_table, int n_table, int num_phys_blocks, int block_size,
-                  int hist_len, float k_scale, float v_scale, float softmax_scale, int Hq, int Hkv,
-                  int G, int Sq, int D, uint16_t* out, cudaStream_t stream) {
-    (void)n_table;
-    (void)D;
+// Shared set-up of both entry points: shared-memory opt-in, tensor maps, launch.
+inline int launch_common(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                         int num_phys_blocks, int block_size, int Hq, int Hkv, int rows_q,
+                         Params prm, dim3 grid, cudaStream_t stream) {
     static std::atomic<uint64_t> smem_done{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -6;
@@ -455,10 +491,20 @@ inline int launch(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_ca
     }
     CUtensorMap tq, tk, tv;
     int rc;
-    if ((rc = encode_map_3d_bf16(&tq, q, kD, Sq, Hq, 64, kTileM))) return rc;
+    if ((rc = encode_map_3d_bf16(&tq, q, kD, rows_q, Hq, 64, kTileM))) return rc;
     const uint64_t planes = static_cast<uint64_t>(num_phys_blocks) * Hkv;
     if ((rc = encode_map_3d_u8(&tk, k_cache, kD, block_size, planes, 128, kTileN))) return rc;
     if ((rc = encode_map_3d_u8(&tv, v_cache, kD, block_size, planes, 128, kTileN))) return rc;
+    return launch_pdl(paged_history_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, prm);
+}
+
+// History only: every query of one sequence sees logical positions [0, hist_len).
+inline int launch(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                  const int32_t* block_table, int n_table, int num_phys_blocks, int block_size,
+                  int hist_len, float k_scale, float v_scale, float softmax_scale, int Hq, int Hkv,
+                  int G, int Sq, int D, uint16_t* out, cudaStream_t stream) {
+    (void)n_table;
+    (void)D;
     Params prm;
     prm.out = out;
     prm.block_table = block_table;
@@ -468,11 +514,39 @@ inline int launch(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_ca
     prm.num_phys_blocks = num_phys_blocks;
     prm.block_size = block_size;
     prm.hist_len = hist_len;
-    prm.n_sub = (hist_len + kTileN - 1) / kTileN;
     prm.c_qk = k_scale * softmax_scale * kLog2e;
     prm.v_scale = v_scale;
-    dim3 grid((Sq + kTileM - 1) / kTileM, Hq);
-    return launch_pdl(paged_history_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, prm);
+    prm.seq_q_start = nullptr;
+    prm.seq_hist = nullptr;
+    prm.table_stride = 0;
+    return launch_common(q, k_cache, v_cache, num_phys_blocks, block_size, Hq, Hkv, Sq, prm,
+                         dim3((Sq + kTileM - 1) / kTileM, Hq), stream);
+}
+
+// Prefill: num_seqs sequences, each seeing its history and its current tokens causally.
+inline int launch_prefill(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                          const int32_t* block_tables, int table_stride, int num_phys_blocks,
+                          int block_size, const int32_t* q_start, const int32_t* hist_lens,
+                          int num_seqs, int total_q, int max_q_len, float k_scale, float v_scale,
+                          float softmax_scale, int Hq, int Hkv, int G, uint16_t* out,
+                          cudaStream_t stream) {
+    if (total_q == 0 || max_q_len == 0) return 0;
+    Params prm;
+    prm.out = out;
+    prm.block_table = block_tables;
+    prm.Sq = total_q;
+    prm.Hkv = Hkv;
+    prm.G = G;
+    prm.num_phys_blocks = num_phys_blocks;
+    prm.block_size = block_size;
+    prm.hist_len = 0;
+    prm.c_qk = k_scale * softmax_scale * kLog2e;
+    prm.v_scale = v_scale;
+    prm.seq_q_start = q_start;
+    prm.seq_hist = hist_lens;
+    prm.table_stride = table_stride;
+    return launch_common(q, k_cache, v_cache, num_phys_blocks, block_size, Hq, Hkv, total_q, prm,
+                         dim3((max_q_len + kTileM - 1) / kTileM, Hq, num_seqs), stream);
 }
 
 }  // namespace paged
