@@ -360,9 +360,20 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tc_fence_after();
             const int kv0 = j * kTileN;
             const int valid = S - kv0;   // keys of this tile that exist
-            const bool full_tile = !kHasBias && valid >= kTileN;
             const float* kb = nullptr;
-            if constexpr (kHasBias) kb = key_bias + static_cast<size_t>(b) * S + kv0;
+            bool full_tile = !kHasBias && valid >= kTileN;
+            if constexpr (kHasBias) {
+                kb = key_bias + static_cast<size_t>(b) * S + kv0;
+                // A complete tile whose 64 bias values of this warp's half are all zero is
+                // computed exactly as without a bias (the common case of right padding: only
+                // the tiles past a sequence's length carry -inf).
+                bool zero = valid >= kTileN;
+                if (zero) {
+                    const int c = col0 + 2 * static_cast<int>(lane_id());
+                    zero = __ldg(kb + c) == 0.f && __ldg(kb + c + 1) == 0.f;
+                }
+                full_tile = __all_sync(0xffffffffu, zero);
+            }
             // score of tile column i in log2 units (scale folded in), -inf where masked;
             // only used on masked tiles (bias or a ragged last tile)
             auto masked_score = [&](float sv, int i) -> float {

@@ -126,3 +126,15 @@ def test_gte_shapes_right_padded_batches(L):
     ref = _oracle(case)
     # rows of padded positions also attend to the valid keys; all rows are compared
     assert_bf16_parity(out, ref, 2, f"gte L={L}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_all_zero_key_bias_equals_no_bias_bitwise(D):
+    """Tiles whose key bias is all zero take the unbiased path: identical results."""
+    c = syn.encoder_case(2, 4, 700, D, seed=77, softmax_scale=D ** -0.5)
+    q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
+    zero = torch.zeros((2, 700), dtype=torch.float32, device=DEV)
+    a = B.attn_encoder_fwd(q, k, v, c.softmax_scale)
+    b = B.attn_encoder_fwd(q, k, v, c.softmax_scale, key_bias=zero)
+    assert B.attn_check() == 0
+    assert torch.equal(a, b)
