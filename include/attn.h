@@ -8,9 +8,10 @@
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers owned by the caller. The library
  *    never frees them and never keeps them after the call returns. The library
- *    allocates no device memory: besides the caller's buffers it only uses one
- *    per-device status word (a static __device__ variable) and kernel
- *    parameters.
+ *    makes no allocation call: besides the caller's buffers it only uses
+ *    static __device__ memory reserved when the library is loaded (one
+ *    per-device status word, and the scratch array of
+ *    attn_gqa_decode_noalloc) and kernel parameters.
  *  - bf16 tensors are passed as `const uint16_t*` holding bf16 bit patterns
  *    (1 sign, 8 exponent, 7 mantissa bits). FP8 caches are `const uint8_t*`
  *    holding E4M3FN codes. All tensors are dense, row-major, contiguous in the
@@ -21,8 +22,8 @@
  *    enqueues work: it returns before the GPU has finished.
  *  - Return value: ATTN_OK or a negative attn_status. A host-side validation
  *    failure enqueues nothing. Errors the device detects (an out-of-range block
- *    table entry, a bounded wait that ran out) are recorded in the per-device
- *    status word and reported by attn_check().
+ *    table entry, a bad sequence descriptor, a bounded wait that ran out) are
+ *    recorded in the per-device status word and reported by attn_check().
  *  - softmax_scale must be finite and > 0. Rows whose every key is masked
  *    produce an all-zero output row.
  *  - Nothing here falls back to another implementation: an unsupported shape

@@ -34,14 +34,39 @@ def sources():
                   if f.endswith((".cu", ".cuh")))
 
 
+def _strip_comments(text: str) -> str:
+    """C / C++ source without its comments and blank lines (string literals kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def source_digest() -> str:
-    """sha256 over the library's CUDA sources and header (identifies a kernel build)."""
+    """sha256 over the library's CUDA sources and header with comments removed: it changes
+    exactly when the code a kernel is built from changes (identifies a kernel build)."""
     import hashlib
     h = hashlib.sha256()
     for path in sources() + [os.path.join(INCLUDE, "attn.h")]:
         h.update(os.path.basename(path).encode())
-        with open(path, "rb") as f:
-            h.update(f.read())
+        with open(path, encoding="utf-8") as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 
