@@ -17,6 +17,8 @@ attention   -- the definition for the entry points (encoder, GQA decode, paged
                split-KV log-sum-exp combine.
 e4m3        -- an FP8 E4M3FN decoder written from the format definition.
 rope        -- rotary position embedding of Q / K rows (both lane pairings).
+precision_model -- float64 replay of the paged FP8 kernel's roundings (hi / lo e4m3
+               splits), used to measure that design choice on the CPU.
 flops       -- the closed-form work counts used for throughput figures.
 """
 
