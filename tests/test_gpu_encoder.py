@@ -138,3 +138,18 @@ def test_all_zero_key_bias_equals_no_bias_bitwise(D):
     b = B.attn_encoder_fwd(q, k, v, c.softmax_scale, key_bias=zero)
     assert B.attn_check() == 0
     assert torch.equal(a, b)
+
+
+def test_general_finite_key_bias():
+    """Arbitrary additive per-key biases (not only 0 / -inf), some tiles all zero."""
+    c = syn.encoder_case(2, 4, 600, 64, seed=78, softmax_scale=0.125)
+    g = torch.Generator().manual_seed(79)
+    kb = (torch.rand((2, 600), generator=g) * 6 - 3).float()
+    kb[:, 128:256] = 0.0                           # one all-zero tile: the unbiased path
+    kb[1, 500:] = float("-inf")
+    q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
+    out = B.attn_encoder_fwd(q, k, v, c.softmax_scale, key_bias=kb.to(DEV))
+    assert B.attn_check() == 0
+    ref = oracle.encoder_attention(to_f64(c.q), to_f64(c.k), to_f64(c.v), c.softmax_scale,
+                                   key_bias=kb.double().numpy())
+    assert_bf16_parity(out, ref, 2, "general key bias")

@@ -89,3 +89,24 @@ def test_bad_sequence_descriptor_is_reported_and_others_are_unaffected():
     out = out.cpu()
     assert torch.equal(out[:, :50], good[:, :50])                 # sequence 0 still computed
     assert torch.count_nonzero(out[:, 50:]) == 0                   # sequence 1 left untouched
+
+
+def test_many_sequences_with_empty_ones_and_block_size_384():
+    g = np.random.default_rng(24)
+    hist = g.integers(0, 900, size=40).tolist()
+    qlen = g.integers(0, 200, size=40).tolist()
+    qlen[3] = qlen[17] = 0                      # sequences with nothing to prefill
+    c = syn.paged_prefill_case(4, 2, 256, 384, hist_lens=hist, q_lens=qlen, seed=25, softmax_scale=1 / 16)
+    out = _run(c)
+    assert B.attn_check() == 0
+    e = rel_l2(to_f64(out), _oracle(c))
+    assert e <= SPLIT_DESIGN_REL_L2, e
+
+
+def test_sequence_that_fills_its_table_row_exactly():
+    c = syn.paged_prefill_case(8, 2, 256, 512, hist_lens=[1536, 1000], q_lens=[512, 24], seed=26,
+                               softmax_scale=1 / 16, spare_blocks=0)
+    assert int((c.block_tables[0] >= 0).sum()) * 512 == 1536 + 512   # every entry used
+    out = _run(c)
+    assert B.attn_check() == 0
+    assert rel_l2(to_f64(out), _oracle(c)) <= SPLIT_DESIGN_REL_L2
