@@ -87,12 +87,13 @@ def load_peaks():
 
 
 def profiled_traffic(kernel_regex: str, workload: str):
-    """DRAM bytes per launch from profiles/dram_traffic.txt, if captured on this build."""
+    """DRAM bytes per launch from profiles/dram_traffic.txt, if captured on a build whose
+    sources for this kernel are the current ones (per-kernel digest)."""
     from online_softmax_attention_flash_b200.build import source_digest
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    digest = source_digest()
+    digest = source_digest(kernel_regex)
     with open(path) as f:
         for line in f:
             parts = line.split()

@@ -20,6 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libattn_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
+_NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+               "-Xcompiler", "-fvisibility=hidden"]
 
 
 def nvcc_path() -> str:
@@ -58,12 +60,30 @@ def _strip_comments(text: str) -> str:
     return "\n".join(line for line in lines if line)
 
 
-def source_digest() -> str:
-    """sha256 over the library's CUDA sources and header with comments removed: it changes
-    exactly when the code a kernel is built from changes (identifies a kernel build)."""
+# The files each kernel's machine code and launch configuration come from (besides the
+# shared PTX / tensor-map / status headers and this file's compiler flags).
+KERNEL_SOURCES = {
+    "encoder_fwd_kernel": ("encoder.cuh", "attn_lib.cu"),   # launch set-up lives in attn_lib.cu
+    "decode_stream_kernel": ("decode.cuh",),
+    "paged_history_kernel": ("paged.cuh",),
+    "rope_qk_kernel": ("rope.cuh",),
+}
+_COMMON_SOURCES = ("ptx.cuh", "tmap.cuh", "status.cuh")
+
+
+def source_digest(kernel: str = None) -> str:
+    """sha256 over source files with comments removed: it changes exactly when the code
+    a build comes from changes. With `kernel` (a key of KERNEL_SOURCES) only the files
+    that kernel is built and launched from count, plus the compiler flags; without it,
+    every CUDA source and the header."""
     import hashlib
     h = hashlib.sha256()
-    for path in sources() + [os.path.join(INCLUDE, "attn.h")]:
+    if kernel is None:
+        paths = sources() + [os.path.join(INCLUDE, "attn.h")]
+    else:
+        paths = [os.path.join(CSRC, f) for f in KERNEL_SOURCES[kernel] + _COMMON_SOURCES]
+        h.update(" ".join(ARCH_FLAGS + _NVCC_FLAGS).encode())
+    for path in paths:
         h.update(os.path.basename(path).encode())
         with open(path, encoding="utf-8") as f:
             h.update(_strip_comments(f.read()).encode())
@@ -82,8 +102,7 @@ def build(force: bool = False, verbose_ptxas: bool = False, out: str = LIB_PATH,
           extra_flags=None) -> str:
     if not force and out == LIB_PATH and up_to_date():
         return out
-    cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
-           "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+    cmd = [nvcc_path(), *ARCH_FLAGS, *_NVCC_FLAGS,
            "-I", INCLUDE, "-I", CSRC,
            "-o", out, os.path.join(CSRC, "attn_lib.cu")]
     if verbose_ptxas:

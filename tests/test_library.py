@@ -115,3 +115,14 @@ def test_rope_validation_rejects_before_any_launch(lib):
     assert f(ctypes.c_void_p(4096 + 8), k, qo, ko, c, s, 1, 1, 8, 64, 0, None) == -4
     assert f(q, k, ctypes.c_void_p(q.value + 256), ko, c, s, 1, 1, 8, 64, 0, None) == -2  # overlap
     assert f(q, k, ko, ko, c, s, 1, 1, 8, 64, 0, None) == -2                    # q_out == k_out
+
+
+def test_source_digest_ignores_comments_and_covers_every_benched_kernel():
+    import bench
+    src = 'int a; // note\n/* block\n comment */ const char* s = "x // y /* z */";\n\n'
+    assert build_mod._strip_comments(src) == 'int a;\n const char* s = "x // y /* z */";'
+    assert build_mod._strip_comments(src) == build_mod._strip_comments(src.replace("note", "other"))
+    benched = set(re.findall(r'self\.kernel_regex = "(\w+)"', open(bench.__file__).read()))
+    assert benched and benched <= set(build_mod.KERNEL_SOURCES)   # each has its own digest
+    for name in benched:
+        assert len(build_mod.source_digest(name)) == 16
