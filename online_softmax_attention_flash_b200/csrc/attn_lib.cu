@@ -1,9 +1,10 @@
 // attn_lib.cu -- the C ABI of libattn_b200.so (declared in include/attn.h).
 //
 // One translation unit: the kernels are header-only (encoder.cuh, decode.cuh,
-// paged.cuh) and included here, so the per-device status word is a single
-// static __device__ variable. Host code validates arguments, encodes TMA
-// tensor maps, and launches on the caller's stream. It allocates nothing.
+// paged.cuh, rope.cuh) and included here, so the per-device status word is a
+// single static __device__ variable. Host code validates arguments, encodes TMA
+// tensor maps, and launches on the caller's stream. It makes no allocation call
+// (the no-alloc decode's scratch is a static __device__ array).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>

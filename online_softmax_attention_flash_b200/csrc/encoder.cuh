@@ -9,15 +9,21 @@
 // How (B200 design, not the pages' SBUF/PSUM one):
 //   * one CTA owns 2 query tiles of 128 rows of one (b, h) and streams the
 //     whole key sequence in 128-key tiles through a TMA ring in shared memory;
-//   * warp 9 (one elected thread) issues tcgen05.mma: S_t = Q_t K^T into a
+//   * warp 17 (one elected thread) issues tcgen05.mma: S_t = Q_t K^T into a
 //     TMEM fp32 accumulator per query tile, then O_t += P_t V with P_t read
-//     back from TMEM (bf16, aliased over S_t) and O_t an fp32 TMEM accumulator;
-//   * warps 0-3 / 4-7 are the softmax warpgroups of query tiles 0 / 1: each
-//     thread owns one query row (one TMEM lane), keeps the running max m and
-//     sum l in fp32 registers, writes P, and rescales its O row in TMEM only
-//     when the row max grew by more than 2^8 (the final O / l uses the same m,
-//     so a stale m is exact);
-//   * warp 8 (one elected thread) is the TMA producer.
+//     back from TMEM (bf16; in its own columns at D = 64, over S_t at D = 128)
+//     and O_t an fp32 TMEM accumulator. At D = 64 it issues in a fixed order per
+//     key tile j -- QK_0(j+1), PV_1(j-1), QK_1(j+1), PV_0(j) -- the order in
+//     which the two softmax warpgroups free their inputs;
+//   * warps 0-7 / 8-15 are the softmax warpgroups of query tiles 0 / 1: a row
+//     (one TMEM lane) is shared by two warps on the same scheduler, 64 S
+//     columns each, which exchange their halves' maxima and sums through
+//     shared memory; each keeps the running max m and sum l in fp32 registers,
+//     writes P, and rescales its half of the O row in TMEM only when the row
+//     max grew by more than 2^8 (the final O / l uses the same m, so a stale m
+//     is exact). At D = 64 one column pair in eight takes 2^x from an FMA-pipe
+//     polynomial instead of the MUFU unit;
+//   * warp 16 (one elected thread) is the TMA producer.
 // The two query tiles ping-pong: while one warpgroup computes exponentials the
 // tensor core runs the other tile's MMAs.
 #pragma once
