@@ -2,8 +2,8 @@
 // tcgen05 (TMEM alloc / MMA / ld / st / commit), fences, and the bounded
 // waits every kernel in this library uses.
 //
-// Nothing here issues a multicast load; every TMA copy reads this GPU's own
-// memory into this CTA's shared memory.
+// Every TMA and bulk copy here reads this GPU's own memory into the issuing
+// CTA's own shared memory, one destination per copy.
 #pragma once
 
 #include <cstdint>
