@@ -83,3 +83,36 @@ def paged_history_emulated(q, k_vals, v_vals, k_scale, v_scale, softmax_scale, s
         pl = e4m3_round(f16_round(ps - ph)) if split_p else np.zeros_like(ph)
         o += (ph + pl) @ V
     return o * v_scale / (p_scale * l[:, None])
+
+
+def bf16_round(x) -> np.ndarray:
+    """Round to bf16 (nearest even), values returned as float64."""
+    a = np.asarray(x, dtype=np.float64).astype(np.float32)
+    bits = a.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
+    return bits.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def encoder_row_emulated(s_row, v, threshold, tile=128):
+    """Online softmax of one query row as the encoder's softmax warps run it.
+
+    s_row [L]: the row's scores already in log2 units (scale * log2 e folded in);
+    v [L, D]. Per 128-key tile: the running max m moves only when the tile's max
+    exceeds it by more than `threshold`; P = 2^(s - m) is rounded to bf16 for the
+    P.V product while the row sum l accumulates the unrounded fp32 values; O is
+    rescaled by 2^(m_old - m_new) when m moves. Returns O / l (before the final
+    bf16 rounding)."""
+    m, l = -np.inf, 0.0
+    o = np.zeros(v.shape[1])
+    for j0 in range(0, s_row.shape[0], tile):
+        s = s_row[j0:j0 + tile]
+        mt = s.max()
+        if mt > m + threshold:
+            alpha = np.exp2(m - mt) if np.isfinite(m) else 0.0
+            l *= alpha
+            o *= alpha
+            m = mt
+        p = f32_round(np.exp2(s - m))
+        l += p.sum()
+        o += bf16_round(p) @ v[j0:j0 + tile]
+    return o / l
