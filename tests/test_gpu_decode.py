@@ -170,3 +170,9 @@ def test_workspace_contents_on_entry_do_not_matter():
     ref = B.attn_gqa_decode(q, k, v, m, case.softmax_scale, case.num_kv_groups)
     assert torch.equal(out.cpu(), ref.cpu())
     assert_bf16_parity(out, _oracle(case), 2, "garbage workspace")
+
+
+def test_large_batch_long_context():
+    """B = 32, 32 Q / 8 KV heads, 16k context, D = 128: many warps per (batch, kv head)."""
+    case = syn.decode_case(32, 32, 8, 16384, 128, seed=76, softmax_scale=128 ** -0.5, min_len=1)
+    assert_bf16_parity(_run(case), _oracle(case), 2, "large batch long context")

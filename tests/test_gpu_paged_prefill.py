@@ -110,3 +110,12 @@ def test_sequence_that_fills_its_table_row_exactly():
     out = _run(c)
     assert B.attn_check() == 0
     assert rel_l2(to_f64(out), _oracle(c)) <= SPLIT_DESIGN_REL_L2
+
+
+def test_pcp_head_shape_16_query_heads_per_kv_head():
+    """The history page's head shape: 32 Q heads sharing 2 KV heads, blocks of 512."""
+    c = syn.paged_prefill_case(32, 2, 256, 512, hist_lens=[2048, 700], q_lens=[300, 129], seed=27,
+                               softmax_scale=1 / 16)
+    out = _run(c)
+    assert B.attn_check() == 0
+    assert rel_l2(to_f64(out), _oracle(c)) <= SPLIT_DESIGN_REL_L2
