@@ -48,13 +48,33 @@ def _as_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
+def _weighted_rows(p, v_head, removed):
+    """num[i] = sum over the keys j that row i keeps of p[i, j] * v[j].
+
+    A removed key (score -inf) takes no part at all, so its V row is never
+    multiplied, not even by p = 0: a non-finite V row at a removed position
+    (an unwritten cache slot) leaves the result finite, while one at a kept
+    position propagates as the definition says.
+    """
+    bad = ~np.isfinite(v_head).all(axis=1)        # keys whose V row holds NaN / inf
+    if not bad.any():
+        return p @ v_head
+    v_fin = np.where(bad[:, None], 0.0, v_head)
+    num = p @ v_fin
+    for j in np.flatnonzero(bad):
+        kept = ~removed[:, j]
+        num[kept] += p[kept, j][:, None] * v_head[j][None, :]
+    return num
+
+
 def _rows_attention(q_rows, k_head, v_head, softmax_scale, mask_rows):
     """Two-pass softmax attention for a block of query rows against one kv head.
 
     q_rows [R, D], k_head/v_head [L, D], mask_rows [R, L] or [1, L] or None.
     Returns (o [R, D], lse [R]) in float64; lse = m + log(l).
     """
-    s = softmax_scale * (q_rows @ k_head.T)                     # scores
+    with np.errstate(invalid="ignore"):                         # NaN rows of removed keys
+        s = softmax_scale * (q_rows @ k_head.T)                 # scores
     if mask_rows is not None:
         s = np.where(np.isneginf(mask_rows), -np.inf, s + mask_rows)
     m = s.max(axis=1) if s.shape[1] > 0 else np.full(s.shape[0], -np.inf)
@@ -62,7 +82,7 @@ def _rows_attention(q_rows, k_head, v_head, softmax_scale, mask_rows):
     m_safe = np.where(live, m, 0.0)
     p = np.exp(s - m_safe[:, None])                             # exp(-inf) = 0 for removed keys
     l = p.sum(axis=1)
-    num = p @ v_head
+    num = _weighted_rows(p, v_head, np.isneginf(s))
     o = np.zeros_like(num)
     nz = l > 0
     o[nz] = num[nz] / l[nz, None]

@@ -225,6 +225,51 @@ def test_fully_masked_row_is_zero_and_lse_neg_inf():
     assert np.array_equal(out[0, 0, 1], np.ones(4)) and abs(lse[0, 0, 1] - 4.0) < 1e-15
 
 
+def test_removed_keys_ignore_nonfinite_k_and_v_rows():
+    # A -inf mask entry removes the key outright: NaN / inf in its K or V row must not reach
+    # the result (truncated problem as the pin), while a NaN V row at a kept key does.
+    r = _rng(12)
+    q = r.standard_normal((2, 4, 1, 8))
+    k = r.standard_normal((2, 2, 20, 8))
+    v = r.standard_normal((2, 2, 20, 8))
+    mask = np.zeros((2, 1, 1, 20))
+    mask[0, ..., [3, 7]] = -np.inf
+    mask[1, ..., 11:] = -np.inf
+    keep0 = [j for j in range(20) if j not in (3, 7)]
+    kk, vv = k.copy(), v.copy()
+    kk[0, :, 3] = np.nan
+    vv[0, :, 3] = np.nan
+    vv[0, :, 7] = np.inf
+    kk[1, :, 15] = np.inf
+    vv[1, :, 12:] = np.nan
+    got = oracle.gqa_decode_attention(q, kk, vv, mask, 1.0, 2)
+    ref0 = brute_attention(q[:1], k[:1, :, keep0], v[:1, :, keep0], 1.0, 2)
+    ref1 = brute_attention(q[1:], k[1:, :, :11], v[1:, :, :11], 1.0, 2)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got[:1] - ref0)) <= 1e-12
+    assert np.max(np.abs(got[1:] - ref1)) <= 1e-12
+    vv[0, :, 5] = np.nan   # kept key
+    assert np.all(np.isnan(oracle.gqa_decode_attention(q, kk, vv, mask, 1.0, 2)[0]))
+
+
+def test_float32_min_fill_keeps_its_keys():
+    # -FLT_MAX (torch.finfo(float32).min, a common mask fill) is finite: a row masked with it
+    # everywhere keeps every key with equal scores (q.k is absorbed), i.e. the mean of V;
+    # next to 0-masked keys those keys get weight e^(-3.4e38) = 0.
+    fmin = float(np.finfo(np.float32).min)
+    r = _rng(13)
+    q = r.standard_normal((1, 2, 1, 8))
+    k = r.standard_normal((1, 1, 12, 8))
+    v = r.standard_normal((1, 1, 12, 8))
+    mask = np.full((1, 1, 1, 12), fmin)
+    got = oracle.gqa_decode_attention(q, k, v, mask, 1.0, 2)
+    assert np.allclose(got[0, :, 0], np.broadcast_to(v[0, 0].mean(axis=0), (2, 8)), atol=1e-15)
+    mask[..., :5] = 0.0
+    got = oracle.gqa_decode_attention(q, k, v, mask, 1.0, 2)
+    ref = brute_attention(q, k[:, :, :5], v[:, :, :5], 1.0, 2)
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
 def test_lse_combine_equals_unsplit_row():
     r = _rng(10)
     D, L = 16, 37
