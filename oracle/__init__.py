@@ -17,6 +17,8 @@ attention   -- the definition for the entry points (encoder, GQA decode, paged
                split-KV log-sum-exp combine.
 e4m3        -- an FP8 E4M3FN decoder written from the format definition.
 rope        -- rotary position embedding of Q / K rows (both lane pairings).
+projection  -- the QKV projection (+ RoPE) and the output projection around the
+               attention core.
 precision_model -- float64 replay of the paged FP8 kernel's roundings (hi / lo e4m3
                splits), used to measure that design choice on the CPU.
 flops       -- the closed-form work counts used for throughput figures.
@@ -33,4 +35,5 @@ from .attention import (  # noqa: F401
 )
 from .e4m3 import e4m3fn_to_float64  # noqa: F401
 from .rope import rope_apply, pair_lanes  # noqa: F401
+from .projection import qkv_projection, qkv_rope_projection, out_projection  # noqa: F401
 from .flops import attention_flops, decode_algorithmic_bytes  # noqa: F401
