@@ -63,6 +63,9 @@ WORKLOADS = {
                      seed0=2200, name="encoder_b1_h16_s2048_d128_x12"),
     "gte": dict(kind="encoder", B=16, H=12, S=512, D=64, scale=0.125, sets=4, seed0=2300,
                 pad=(128, 512), name="gte_b16_h12_s512_d64_rightpad_128_512"),
+    # the headline decode with 8 query heads per kv head (same K/V bytes, 4x the heads)
+    "decode_g8": dict(kind="decode", B=8, Hq=64, Hkv=8, S=4096, D=256, scale=1.0, sets=4,
+                      seed0=2900, name="gqa_decode_b8_64q_8kv_d256_ctx4096"),
     "decode_d512": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=512, scale=512 ** -0.5,
                         sets=4, seed0=2400, name="gqa_decode_b8_16q_8kv_d512_ctx4096"),
     "decode_window": dict(kind="decode", B=8, Hq=16, Hkv=8, S=4096, D=256, scale=1.0, sets=4,
@@ -72,6 +75,11 @@ WORKLOADS = {
     "paged_prefill": dict(kind="prefill", Hq=32, Hkv=2, D=256, BS=512, n_seqs=8,
                           hist=(4096, 16384), qlen=(512, 2048), scale=1.0 / 16, sets=1,
                           seed0=2700, name="paged_prefill_8seq_32q_2kv_d256_hist4k_16k_q512_2k_fp8"),
+    # the whole attention block of a ViT-L layer: QKV projection with RoPE in its epilogue,
+    # attention, output projection (random-init Linear weights), 24 layers
+    "vitl_block": dict(kind="block", B=1, H=16, S=2048, D=64, C=1024, scale=0.125, sets=24,
+                       seed0=2800, interleaved=True,
+                       name="vitl_attention_block_b1_s2048_c1024_h16_d64_x24layers"),
     # the RoPE prologue of the ViT-L encoder (V-JEPA2 pairs lanes 2j, 2j+1), 24 layers
     "rope_vitl": dict(kind="rope", B=1, H=16, S=2048, D=64, sets=24, seed0=2600, interleaved=True,
                       name="rope_qk_vitl_b1_h16_s2048_d64_interleaved_x24layers"),
@@ -89,9 +97,9 @@ def load_peaks():
 def profiled_traffic(kernel_regex: str, workload: str):
     """DRAM bytes per launch from profiles/dram_traffic.txt, if captured on a build whose
     sources for this kernel are the current ones (per-kernel digest)."""
-    from online_softmax_attention_flash_b200.build import source_digest
+    from online_softmax_attention_flash_b200.build import KERNEL_SOURCES, source_digest
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel_regex not in KERNEL_SOURCES:
         return None
     digest = source_digest(kernel_regex)
     with open(path) as f:
@@ -406,6 +414,92 @@ class RopeWork:
         return 4.0 * S * D * 2 + 2.0 * S * (D // 2) * 4, "the q and k rows of one head"
 
 
+class BlockWork:
+    """attn_qkv_rope_proj -> attn_encoder_fwd -> attn_out_proj for 24 layers (distinct inputs
+    and random-init weights per layer). All three kernels are bf16 tensor-core work: the
+    roofline is the block's algorithmic flops over its time against the bf16 peak."""
+
+    def __init__(self, cfg, device):
+        import torch
+        from online_softmax_attention_flash_b200 import inputs as syn
+        self.cfg = cfg
+        B, S, C, H, D = cfg["B"], cfg["S"], cfg["C"], cfg["H"], cfg["D"]
+        self.host = [syn.projection_case(B, S, C, H, D, seed=cfg["seed0"] + i)
+                     for i in range(cfg["sets"])]
+        self.h_tables = syn.rope_tables(S, D)
+        self.tables = tuple(t.to(device) for t in self.h_tables)
+        self.dev = [dict(x=c.x.to(device), w_qkv=c.w_qkv.to(device), b_qkv=c.b_qkv.to(device),
+                         w_o=c.w_o.to(device), b_o=c.b_o.to(device)) for c in self.host]
+        shp = (B, H, S, D)
+        self.bufs = [dict(q=torch.empty(shp, dtype=torch.bfloat16, device=device),
+                          k=torch.empty(shp, dtype=torch.bfloat16, device=device),
+                          v=torch.empty(shp, dtype=torch.bfloat16, device=device),
+                          o=torch.empty(shp, dtype=torch.bfloat16, device=device),
+                          y=torch.empty((B, S, C), dtype=torch.float32, device=device))
+                     for _ in self.host]
+        HD = H * D
+        self.flops_qkv = 2.0 * B * S * C * 3 * HD
+        self.flops_attn = 4.0 * B * H * S * S * D
+        self.flops_out = 2.0 * B * S * HD * C
+        self.flops_per_launch = (self.flops_qkv + self.flops_attn + self.flops_out) / 3
+        self.launches_per_step = 3 * cfg["sets"]
+        self.work_per_step = (self.flops_qkv + self.flops_attn + self.flops_out) * cfg["sets"]
+        self.unit, self.bound = "TFLOP/s", "tensor"
+        self.kernel_regex = "proj_gemm_kernel|encoder_fwd_kernel"
+        self.peak_ratio = 1.0
+        self.dtype = "bf16"
+
+    def _layer(self, d, bf, stream):
+        from online_softmax_attention_flash_b200 import binding as Bd
+        c = self.cfg
+        Bd.attn_qkv_rope_proj(d["x"], d["w_qkv"], d["b_qkv"], c["H"], c["D"], *self.tables,
+                              interleaved=c["interleaved"], q=bf["q"], k=bf["k"], v=bf["v"],
+                              stream=stream)
+        Bd.attn_encoder_fwd(bf["q"], bf["k"], bf["v"], c["scale"], out=bf["o"], stream=stream)
+        Bd.attn_out_proj(bf["o"], d["w_o"], d["b_o"], y=bf["y"], stream=stream)
+
+    def step(self, stream=None):
+        for d, bf in zip(self.dev, self.bufs):
+            self._layer(d, bf, stream)
+
+    def rate(self, work, seconds):
+        return work / seconds / 1e12
+
+    def e2e_setup(self):
+        import torch
+        self.h_x = [c.x.pin_memory() for c in self.host]
+        self.h_y = [torch.empty_like(bf["y"], device="cpu").pin_memory() for bf in self.bufs]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_x)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_y)
+
+    def e2e_step(self, stream):
+        for hx, hy, d, bf in zip(self.h_x, self.h_y, self.dev, self.bufs):
+            d["x"].copy_(hx, non_blocking=True)
+            self._layer(d, bf, stream)
+            hy.copy_(bf["y"], non_blocking=True)
+
+    def oracle_sample(self, step_idx, rows=256):
+        import oracle
+        c = self.host[step_idx % len(self.host)]
+        cfg = self.cfg
+        S, C, H, D = cfg["S"], cfg["C"], cfg["H"], cfg["D"]
+        h = step_idx % H
+        # one head's q, k, v for every token, its attention for `rows` queries, and the
+        # out-projection of those rows (this head's share of the sum)
+        sel = np.concatenate([np.arange(w * H * D + h * D, w * H * D + (h + 1) * D) for w in range(3)])
+        x = c.x.double().numpy()
+        q, k, v = oracle.qkv_rope_projection(x, c.w_qkv.double().numpy()[sel],
+                                             c.b_qkv.double().numpy()[sel], 1, D,
+                                             *(t.double().numpy() for t in self.h_tables),
+                                             "interleaved" if cfg["interleaved"] else "half")
+        r0 = (step_idx * rows) % (S - rows + 1)
+        rr = np.arange(r0, r0 + rows)
+        o = oracle.encoder_attention(q, k, v, cfg["scale"], rows=rr)
+        oracle.out_projection(o, c.w_o.double().numpy()[:, h * D:(h + 1) * D], None)
+        flops = 2.0 * S * C * 3 * D + 4.0 * rows * S * D + 2.0 * rows * D * C
+        return flops, f"one head of one layer: q/k/v of all {S} tokens, {rows} query rows"
+
+
 def rope_host_case(cfg, i):
     from online_softmax_attention_flash_b200 import inputs as syn
     import torch
@@ -554,13 +648,13 @@ class PrefillWork(PagedWork):
 # steps captured per CUDA graph for the timed region (decode rotates 4 input sets)
 GRAPH_STEPS = {"vitl": 1, "tiny": 20, "dinov3": 20, "decode": 4, "paged": 1, "vitl8k": 1,
                "enc_d128": 1, "gte": 4, "decode_d512": 4, "decode_window": 4, "rope_vitl": 1,
-               "paged_prefill": 1}
+               "paged_prefill": 1, "vitl_block": 1, "decode_g8": 4}
 
 
 def make_work(name, device):
     cfg = WORKLOADS[name]
     return {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork,
-            "rope": RopeWork, "prefill": PrefillWork}[cfg["kind"]](cfg, device)
+            "rope": RopeWork, "prefill": PrefillWork, "block": BlockWork}[cfg["kind"]](cfg, device)
 
 
 # --------------------------------------------------------------------- oracle
@@ -615,7 +709,7 @@ def make_work_host_only(name):
     """Host-side inputs only (the oracle arm never touches a GPU)."""
     cfg = WORKLOADS[name]
     cls = {"encoder": EncoderWork, "decode": DecodeWork, "paged": PagedWork,
-           "rope": RopeWork, "prefill": PrefillWork}[cfg["kind"]]
+           "rope": RopeWork, "prefill": PrefillWork, "block": BlockWork}[cfg["kind"]]
     obj = cls.__new__(cls)
     obj.cfg = cfg
     from online_softmax_attention_flash_b200 import inputs as syn
@@ -628,6 +722,11 @@ def make_work_host_only(name):
     elif cfg["kind"] == "prefill":
         obj.host = [prefill_host_case(cfg)]
         obj.unit = "TFLOP/s"
+    elif cfg["kind"] == "block":
+        obj.host = [syn.projection_case(cfg["B"], cfg["S"], cfg["C"], cfg["H"], cfg["D"],
+                                        seed=cfg["seed0"] + i) for i in range(cfg["sets"])]
+        obj.h_tables = syn.rope_tables(cfg["S"], cfg["D"])
+        obj.unit = "TFLOP/s"
     elif cfg["kind"] == "rope":
         obj.host = [rope_host_case(cfg, i) for i in range(cfg["sets"])]
         obj.h_tables = syn.rope_tables(cfg["S"], cfg["D"])
@@ -639,29 +738,28 @@ def make_work_host_only(name):
     return obj
 
 
-def run_product(args, info):
+# the other configurations the headline metric is quoted on, measured in the same default run
+# (1 GPU): steps per config, chosen so each timed region is about a tenth of a second or more
+CONFIG_STEPS = {"tiny": 2000, "dinov3": 2000, "decode": 2000, "paged": 60}
+
+
+def time_work(work, workload, steps, warmup, info, device, stream, use_graph):
+    """Warm up, then time `steps` steps (CUDA-graph replays of the same C-ABI launches) with
+    CUDA events on the launching stream between barriers; clocks sampled meanwhile."""
     import torch
     from online_softmax_attention_flash_b200 import binding as Bd
     from online_softmax_attention_flash_b200 import dist as D
-
-    torch.cuda.set_device(info.local_rank)
-    device = torch.device("cuda", info.local_rank)
-    Bd.load_library()
-    work = make_work(args.workload, device)
-    stream = torch.cuda.current_stream(device)
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         work.step(stream)
     torch.cuda.synchronize(device)
     st = Bd.attn_check(stream)
     if st != 0:
-        raise RuntimeError(f"device status after warm-up: {Bd.STATUS.get(st, st)}")
-
+        raise RuntimeError(f"{workload}: device status after warm-up: {Bd.STATUS.get(st, st)}")
     # The timed region replays CUDA graphs that capture the same C-ABI launches (n steps per
     # graph), so per-call host overhead (Python, ctypes, tensor-map encoding) is not timed.
-    n_graph = math.gcd(GRAPH_STEPS[args.workload], args.steps) if args.graph else 1
+    n_graph = math.gcd(GRAPH_STEPS[workload], steps) if use_graph else 1
     graph = None
-    if args.graph:
+    if use_graph:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             for _ in range(n_graph):
@@ -669,7 +767,7 @@ def run_product(args, info):
         for _ in range(2):
             graph.replay()
         torch.cuda.synchronize(device)
-    replays = args.steps // n_graph
+    replays = steps // n_graph
     sampler = ClockSampler(gpu_smi_id(device))
     sampler.start()
     time.sleep(0.2)
@@ -692,18 +790,17 @@ def run_product(args, info):
     del graph
     st = Bd.attn_check(stream)
     if st != 0:
-        raise RuntimeError(f"device status after timing: {Bd.STATUS.get(st, st)}")
-    max_ms = D.max_over_ranks(total_ms, info, device)
+        raise RuntimeError(f"{workload}: device status after timing: {Bd.STATUS.get(st, st)}")
+    return total_ms, step_ms, clocks, launch_mode
 
-    work_all = work.work_per_step * args.steps * info.world_size
-    value = work.rate(work_all, max_ms / 1e3)
 
-    # roofline of the dominant kernel: algorithmic work per launch / mean launch time
+def roofline_of(work, workload, total_ms, steps):
+    """Dominant kernel: algorithmic work per launch / mean launch time against the peak."""
     peaks, peak_src = load_peaks()
-    per_launch_ms = total_ms / (args.steps * work.launches_per_step)
+    per_launch_ms = total_ms / (steps * work.launches_per_step)
     if work.bound == "hbm":
         # decode: one call = scan + stream + combine; achieved counts the whole call's time
-        per_call_ms = total_ms / args.steps
+        per_call_ms = total_ms / steps
         achieved = work.work_per_step / (per_call_ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         peak_name = "hbm_gbs"
@@ -714,10 +811,60 @@ def run_product(args, info):
         peak = float(peaks[peak_name]) * work.peak_ratio
         if work.peak_ratio != 1.0:
             peak_name += f" x {work.peak_ratio:g} (fp8/bf16 nominal ratio)"
-    roofline = {"bound": work.bound, "achieved": achieved, "peak": peak, "unit": work.unit,
-                "frac": achieved / peak,
-                "traffic": profiled_traffic(work.kernel_regex, args.workload),
-                "peak_source": f"{peak_src} ({peak_name})", "kernel": work.kernel_regex}
+    return {"bound": work.bound, "achieved": achieved, "peak": peak, "unit": work.unit,
+            "frac": achieved / peak, "traffic": profiled_traffic(work.kernel_regex, workload),
+            "peak_source": f"{peak_src} ({peak_name})", "kernel": work.kernel_regex}
+
+
+def step_stats(step_ms):
+    s_sorted = sorted(step_ms)
+    return {"min": s_sorted[0], "median": statistics.median(step_ms),
+            "mean": statistics.fmean(step_ms),
+            "p90": s_sorted[min(len(s_sorted) - 1, int(0.9 * len(s_sorted)))],
+            "max": s_sorted[-1]}
+
+
+def measure_config(name, args, info, device, stream):
+    """One more configuration, measured like the headline (own clocks, own roofline), with a
+    short oracle sample on the host cores beside it."""
+    import torch
+    work = make_work(name, device)
+    steps = CONFIG_STEPS[name]
+    total_ms, step_ms, clocks, mode = time_work(work, name, steps, 5, info, device, stream,
+                                                args.graph)
+    entry = {"workload": WORKLOADS[name]["name"],
+             "value": work.rate(work.work_per_step * steps, total_ms / 1e3), "unit": work.unit,
+             "ms_per_step": total_ms / steps, "steps": steps, "launch": mode,
+             "step_ms": step_stats(step_ms), "roofline": roofline_of(work, name, total_ms, steps),
+             "clocks": clocks, "dtype": work.dtype,
+             "gpu_launches": steps * work.launches_per_step}
+    if not args.no_cpu_baseline:
+        rate, secs, sample, n = cpu_oracle_run(work, args.config_cpu_budget)
+        entry["cpu_baseline"] = {"value": rate, "unit": work.unit, "cores": cores(),
+                                 "kind": "oracle",
+                                 "sample": f"{n} samples of {sample} ({secs:.1f} s of fp64 NumPy)"}
+    del work
+    torch.cuda.empty_cache()
+    return entry
+
+
+def run_product(args, info):
+    import torch
+    from online_softmax_attention_flash_b200 import binding as Bd
+    from online_softmax_attention_flash_b200 import dist as D
+
+    torch.cuda.set_device(info.local_rank)
+    device = torch.device("cuda", info.local_rank)
+    Bd.load_library()
+    work = make_work(args.workload, device)
+    stream = torch.cuda.current_stream(device)
+
+    total_ms, step_ms, clocks, launch_mode = time_work(work, args.workload, args.steps, args.warmup,
+                                                       info, device, stream, args.graph)
+    max_ms = D.max_over_ranks(total_ms, info, device)
+    work_all = work.work_per_step * args.steps * info.world_size
+    value = work.rate(work_all, max_ms / 1e3)
+    roofline = roofline_of(work, args.workload, total_ms, args.steps)
 
     # end to end through the public API with host buffers
     work.e2e_setup()
@@ -737,6 +884,12 @@ def run_product(args, info):
            "unit": work.unit, "h2d_bytes_per_step": int(work.h2d),
            "d2h_bytes_per_step": int(work.d2h), "steps": e2e_steps}
 
+    dtype, launches = work.dtype, args.steps * work.launches_per_step
+    # the remaining configurations of the metric, 1 GPU, same run (default workload only)
+    configs = None
+    if info.world_size == 1 and args.workload == "vitl" and args.configs:
+        configs = {n: measure_config(n, args, info, device, stream) for n in CONFIG_STEPS}
+
     if not info.is_main:
         return 0
     cpu = None
@@ -745,27 +898,25 @@ def run_product(args, info):
         cpu = {"value": rate, "unit": work.unit, "cores": cores(), "kind": "oracle",
                "sample": f"{n} samples of {sample} ({secs:.1f} s of fp64 NumPy)"}
     cfg = WORKLOADS[args.workload]
-    s_sorted = sorted(step_ms)
     line = {
         "metric": METRIC, "value": value, "unit": work.unit, "n_gpus": info.world_size,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": work.dtype,
-        "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype, "data": "synthetic",
         "config": {"workload": cfg["name"],
                    **{k: v for k, v in cfg.items() if k not in ("kind", "name", "seed0")},
                    "l2": ("inputs larger than L2: distinct input sets rotate across calls"
                           if cfg["sets"] > 1 or cfg["kind"] in ("paged", "prefill") else "inputs fit in L2"),
                    "parallelism": f"replicas x{info.world_size}", "launch": launch_mode},
-        "step_ms": {"min": s_sorted[0], "median": statistics.median(step_ms),
-                    "mean": statistics.fmean(step_ms),
-                    "p90": s_sorted[min(len(s_sorted) - 1, int(0.9 * len(s_sorted)))],
-                    "max": s_sorted[-1]},
+        "step_ms": step_stats(step_ms),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps * work.launches_per_step,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
+    if configs is not None:
+        line["configs"] = configs
     print(json.dumps(line), flush=True)
     return 0
 
@@ -782,12 +933,17 @@ def main(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", dest="graph", action="store_false",
                    help="time eager calls instead of CUDA-graph replays")
+    p.add_argument("--no-configs", dest="configs", action="store_false",
+                   help="skip the other configurations of the default run")
+    p.add_argument("--config-cpu-budget", type=float, default=3.0,
+                   help="seconds of oracle work per additional configuration")
     args = p.parse_args(argv)
     defaults = {"vitl": (1000, 20), "tiny": (2000, 20), "dinov3": (2000, 20),
                 "decode": (2000, 20), "paged": (100, 5), "vitl8k": (400, 10),
                 "enc_d128": (1000, 20), "gte": (2000, 20), "decode_d512": (2000, 20),
                 "decode_window": (2000, 20), "rope_vitl": (1000, 20),
-                "paged_prefill": (30, 5)}[args.workload]
+                "paged_prefill": (30, 5), "vitl_block": (300, 10),
+                "decode_g8": (2000, 20)}[args.workload]
     if args.steps is None:
         args.steps = defaults[0]
     if args.warmup is None:

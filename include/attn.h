@@ -71,7 +71,8 @@ typedef enum attn_status {
  *   B, H >= 1; S >= 1; D in {64, 128}.
  *   softmax_scale: finite, > 0 (1/sqrt(D) for the ViT encoders).
  *   key_bias     : NULL, or [B, S] fp32 additive bias added to every query's
- *                  score for key j of batch entry b (0 keep, -inf drop).
+ *                  score for key j of batch entry b (0 keep, -inf drop; any
+ *                  finite value, -FLT_MAX included, keeps the key).
  *
  * Every query row attends to all S keys (no causal mask). Accumulation is fp32;
  * out is rounded to bf16 (round-to-nearest-even).
@@ -101,7 +102,9 @@ ATTN_API size_t attn_gqa_decode_workspace_size(int B, int Hq, int Hkv, int S_ctx
  *   q         : [B, Hq, 1, D] bf16
  *   k, v      : [B, Hkv, S_ctx, D] bf16
  *   attn_mask : NULL (no mask), or [B, 1, 1, S_ctx] fp32 additive (0 keep,
- *               -inf drop). A -inf entry removes the key whatever its K holds.
+ *               -inf drop). A -inf entry removes the key whatever its K and V
+ *               rows hold (even NaN); any finite value, -FLT_MAX included,
+ *               keeps the key with that additive score.
  *   out       : [B, Hq, 1, D] bf16
  *   Hq == Hkv * num_kv_groups; query head h reads kv head h / num_kv_groups.
  *   D in {128, 256, 512}; S_ctx >= 1 (no multiple-of-128 requirement).
@@ -141,7 +144,8 @@ ATTN_API int attn_gqa_decode(const uint16_t* q, const uint16_t* k, const uint16_
  *   exceed ATTN_NOALLOC_SCRATCH_BYTES; larger problems are rejected with
  *   ATTN_ERR_WORKSPACE before anything is enqueued.
  *   Set-up: the first call on a device looks up the scratch array's device
- *   address on the current device (once per device). Make that first call
+ *   address on the current device (once per device; again only if the device's
+ *   context was re-created, e.g. after cudaDeviceReset). Make that first call
  *   outside any stream capture.
  *   Sharing: all calls on a device use the same scratch array, which keeps the
  *   previous call's contents (nothing in it needs to start at zero). Calls that
@@ -266,6 +270,58 @@ ATTN_API int attn_paged_prefill(const uint16_t* q, const uint8_t* k_cache, const
 ATTN_API int attn_rope_qk(const uint16_t* q, const uint16_t* k, uint16_t* q_out, uint16_t* k_out,
                           const float* cos_table, const float* sin_table,
                           int B, int H, int S, int D, int interleaved, void* stream);
+
+/*
+ * attn_qkv_rope_proj -- the QKV projection in front of the encoder attention,
+ * with RoPE applied to Q and K in the same kernel.
+ *
+ * Defined by: "V-JEPA2 ViT-L Encoder NKI Kernels for AWS Trainium2", section
+ * "Repository layout" (the attention block K2: QKV projection + RoPE, then the
+ * attention inner, then the output projection; LayerNorm affines are folded into
+ * the weights, so the projection is a plain affine map) and
+ * "vit-encoder-neuron-kernels", section "Kernels" (both RoPE lane pairings):
+ *     t = x W_qkv^T + b_qkv,   t [B, S, 3 H D]
+ * column block 0 of t is Q, block 1 K, block 2 V; column h D + d of a block is
+ * head h, lane d. Q and K are then rotated exactly as attn_rope_qk rotates them
+ * (in fp32, before the single rounding to bf16); V is not rotated.
+ *
+ *   x          : [B, S, C] bf16 (the block's normalised input)
+ *   w_qkv      : [3 H D, C] bf16 (a torch.nn.Linear weight: out x in)
+ *   b_qkv      : NULL or [3 H D] fp32
+ *   cos_table, sin_table : NULL (no rotation) or [S, D/2] fp32 each, row s for
+ *                token s; interleaved selects the pairing as in attn_rope_qk
+ *   q, k, v    : [B, H, S, D] bf16 outputs, ready for attn_encoder_fwd
+ *   B, S, H >= 1; D in {64, 128}; C a multiple of 64; H * D a multiple of 128.
+ * fp32 accumulation on the tensor cores. All pointers 16-byte aligned; the
+ * caller owns every buffer.
+ * Errors: ATTN_ERR_NULL (a table without the other), ATTN_ERR_SHAPE,
+ * ATTN_ERR_UNSUPPORTED, ATTN_ERR_ALIGN, ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_qkv_rope_proj(const uint16_t* x, const uint16_t* w_qkv, const float* b_qkv,
+                                const float* cos_table, const float* sin_table, int interleaved,
+                                int B, int S, int C, int H, int D,
+                                uint16_t* q, uint16_t* k, uint16_t* v, void* stream);
+
+/*
+ * attn_out_proj -- the output projection behind the encoder attention.
+ *
+ * Defined by: "V-JEPA2 ViT-L Encoder NKI Kernels for AWS Trainium2", section
+ * "Repository layout" (K2 outer: the out-projection of the attention block):
+ *     y[b, s, :] = a[b, s, :] W_o^T + b_o,   a[b, s, h D + d] = o[b, h, s, d]
+ * (the heads side by side, read straight from the attention layout).
+ *
+ *   o     : [B, H, S, D] bf16 (attn_encoder_fwd's output)
+ *   w_o   : [C_out, H D] bf16 (a torch.nn.Linear weight)
+ *   b_o   : NULL or [C_out] fp32
+ *   y     : [B, S, C_out] fp32 (kept in fp32: it is added to the fp32 residual
+ *           stream)
+ *   B, S, H >= 1; D in {64, 128}; C_out a multiple of 128.
+ * All pointers 16-byte aligned; the caller owns every buffer.
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_UNSUPPORTED, ATTN_ERR_ALIGN,
+ * ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_out_proj(const uint16_t* o, const uint16_t* w_o, const float* b_o,
+                           int B, int S, int H, int D, int C_out, float* y, void* stream);
 
 /*
  * attn_check -- synchronise `stream`, then return and clear the first error the

@@ -41,6 +41,8 @@ SIGNATURES = [
     ("attn_paged_prefill", _I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _F, _F, _F, _I, _I,
                                 _I, _I, _P, _P]),
     ("attn_rope_qk", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    ("attn_qkv_rope_proj", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    ("attn_out_proj", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     ("attn_check", _I, [_P]),
     ("attn_status_string", ctypes.c_char_p, [_I]),
     ("attn_version", _I, []),
@@ -269,3 +271,50 @@ def attn_rope_qk(q, k, cos_table, sin_table, interleaved: bool = False, q_out=No
                           _ptr(sin_table), B, H, S, D, 1 if interleaved else 0, _stream_ptr(stream))
     _raise_if(st, "attn_rope_qk")
     return q_out, k_out
+
+
+def attn_qkv_rope_proj(x, w_qkv, b_qkv, H: int, D: int, cos_table=None, sin_table=None,
+                       interleaved: bool = False, q=None, k=None, v=None, stream=None):
+    """x [B, S, C] bf16, w_qkv [3 H D, C] bf16, b_qkv [3 H D] fp32 or None; optional RoPE
+    tables [S, D/2] fp32. Returns (q, k, v), each [B, H, S, D] bf16, q and k rotated."""
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    B, S, C = x.shape
+    _need(w_qkv, "w_qkv", torch.bfloat16, (3 * H * D, C))
+    if b_qkv is not None:
+        _need(b_qkv, "b_qkv", torch.float32, (3 * H * D,))
+    if (cos_table is None) != (sin_table is None):
+        raise ValueError("pass both RoPE tables or neither")
+    if cos_table is not None:
+        _need(cos_table, "cos_table", torch.float32, (S, D // 2))
+        _need(sin_table, "sin_table", torch.float32, (S, D // 2))
+    shape = (B, H, S, D)
+    q = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if v is None else v
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, shape)
+    st = lib.attn_qkv_rope_proj(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(cos_table),
+                                _ptr(sin_table), 1 if interleaved else 0, B, S, C, H, D, _ptr(q),
+                                _ptr(k), _ptr(v), _stream_ptr(stream))
+    _raise_if(st, "attn_qkv_rope_proj")
+    return q, k, v
+
+
+def attn_out_proj(o, w_o, b_o=None, y=None, stream=None):
+    """o [B, H, S, D] bf16, w_o [C_out, H D] bf16, b_o [C_out] fp32 or None -> y [B, S, C_out] fp32."""
+    lib = load_library()
+    _need(o, "o", torch.bfloat16)
+    B, H, S, D = o.shape
+    _need(w_o, "w_o", torch.bfloat16)
+    C_out = w_o.shape[0]
+    if w_o.dim() != 2 or w_o.shape[1] != H * D:
+        raise ValueError("w_o must be [C_out, H * D]")
+    if b_o is not None:
+        _need(b_o, "b_o", torch.float32, (C_out,))
+    y = torch.empty((B, S, C_out), dtype=torch.float32, device=o.device) if y is None else y
+    _need(y, "y", torch.float32, (B, S, C_out))
+    st = lib.attn_out_proj(_ptr(o), _ptr(w_o), _ptr(b_o), B, S, H, D, C_out, _ptr(y),
+                           _stream_ptr(stream))
+    _raise_if(st, "attn_out_proj")
+    return y

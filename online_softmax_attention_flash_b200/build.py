@@ -67,6 +67,7 @@ KERNEL_SOURCES = {
     "decode_stream_kernel": ("decode.cuh",),
     "paged_history_kernel": ("paged.cuh",),
     "rope_qk_kernel": ("rope.cuh",),
+    "proj_gemm_kernel": ("proj.cuh", "attn_lib.cu"),
 }
 _COMMON_SOURCES = ("ptx.cuh", "tmap.cuh", "status.cuh")
 

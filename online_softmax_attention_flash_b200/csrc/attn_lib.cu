@@ -19,6 +19,7 @@
 #include "decode.cuh"
 #include "encoder.cuh"
 #include "paged.cuh"
+#include "proj.cuh"
 #include "rope.cuh"
 #include "tmap.cuh"
 
@@ -72,16 +73,41 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SC
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};   // context the cached address belongs to
 
-// Device address of g_noalloc_scratch on the current device (looked up once per device).
+// The current driver context (the runtime's primary context of the current device once
+// any runtime call has run on it), through the driver entry point the runtime exposes.
+CUcontext current_context() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    static GetCurrent fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCurrent>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (fn) fn(&ctx);
+    return ctx;
+}
+
+// Device address of g_noalloc_scratch on the current device. It is looked up once per
+// device and context: after cudaDeviceReset the module is loaded again in a new primary
+// context, possibly at another address, so a change of context repeats the look-up.
 int noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    // No context current on this thread yet (ctx == NULL) also repeats the look-up, which
+    // makes the device's primary context current; the context is read again after it.
+    const CUcontext ctx = current_context();
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
+    if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = current_context();
     }
     *out = g_scratch_ptr[dev];
     return ATTN_OK;
@@ -250,6 +276,37 @@ int attn_rope_qk(const uint16_t* q, const uint16_t* k, uint16_t* q_out, uint16_t
         return ATTN_ERR_SHAPE;
     return attn::rope::launch(q, k, q_out, k_out, cos_table, sin_table, B, H, S, D,
                               interleaved != 0, static_cast<cudaStream_t>(stream));
+}
+
+int attn_qkv_rope_proj(const uint16_t* x, const uint16_t* w_qkv, const float* b_qkv,
+                       const float* cos_table, const float* sin_table, int interleaved, int B,
+                       int S, int C, int H, int D, uint16_t* q, uint16_t* k, uint16_t* v,
+                       void* stream) {
+    if (!x || !w_qkv || !q || !k || !v) return ATTN_ERR_NULL;
+    if ((cos_table == nullptr) != (sin_table == nullptr)) return ATTN_ERR_NULL;
+    if (B < 1 || S < 1 || C < 1 || H < 1 || (interleaved != 0 && interleaved != 1))
+        return ATTN_ERR_SHAPE;
+    if ((D != 64 && D != 128) || C % 64 || (H * D) % 128 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(H) * D > (1 << 20) || C > (1 << 20)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        (b_qkv && !aligned16(b_qkv)) || (cos_table && (!aligned16(cos_table) || !aligned16(sin_table))))
+        return ATTN_ERR_ALIGN;
+    const int rope = cos_table ? (interleaved ? 2 : 1) : 0;
+    return attn::proj::launch_qkv(x, w_qkv, b_qkv, cos_table, sin_table, rope, B, S, C, H, D, q, k,
+                                  v, static_cast<cudaStream_t>(stream));
+}
+
+int attn_out_proj(const uint16_t* o, const uint16_t* w_o, const float* b_o, int B, int S, int H,
+                  int D, int C_out, float* y, void* stream) {
+    if (!o || !w_o || !y) return ATTN_ERR_NULL;
+    if (B < 1 || S < 1 || H < 1 || C_out < 1) return ATTN_ERR_SHAPE;
+    if ((D != 64 && D != 128) || C_out % 128 || B > 65535 || C_out / 128 > 65535)
+        return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(H) * D > (1 << 20)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(o) || !aligned16(w_o) || !aligned16(y) || (b_o && !aligned16(b_o)))
+        return ATTN_ERR_ALIGN;
+    return attn::proj::launch_out(o, w_o, b_o, B, S, H, D, C_out, y,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

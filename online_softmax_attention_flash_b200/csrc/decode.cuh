@@ -227,8 +227,14 @@ decode_scan_kernel(const float* __restrict__ mask, int S_ctx, Workspace ws) {
 #pragma unroll
         for (int kk = 0; kk < kSubKeys; ++kk) {
             const int key = st * kSubKeys + kk;
+            // liveness is decided on the stored value: only -inf removes a key. A finite mask
+            // value is clamped after the change to log2 units, so that large negative fills
+            // (e.g. -FLT_MAX) stay finite and keep their key, as the definition says.
             float x = -INFINITY;
-            if (st < n_sub && key < S_ctx) x = mask ? mask[static_cast<size_t>(b) * S_ctx + key] * kLog2e : 0.f;
+            if (st < n_sub && key < S_ctx) {
+                const float mraw = mask ? mask[static_cast<size_t>(b) * S_ctx + key] : 0.f;
+                if (mraw != -INFINITY) x = fmaxf(mraw * kLog2e, -FLT_MAX);
+            }
             mv[kk] = x;
             live |= (x != -INFINITY);
         }
@@ -436,11 +442,14 @@ decode_stream_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict_
     for (int u = 0; u < n; ++u) {
         const int st = u % S;
         const uint32_t ph = (u / S) & 1;
-        ok = mbar_wait(&bar[2 * st], ph, abort_flag);
+        ok = mbar_wait_warp(&bar[2 * st], ph, abort_flag);
         if (!ok) break;
         const int4 inf = info[st];
-        const int rows = inf.y;
         const float mv = smask[st * kSubKeys + kk_me];
+        // keys of this sub-tile that take part: bit kk * kBase is set when key kk is live
+        // (mask not -inf; keys past S_ctx carry -inf). Taken now, because the stage's mask
+        // slot is refilled before the P.V step below.
+        const uint32_t live_bits = __ballot_sync(0xffffffffu, mv != -INFINITY);
         if (inf.z != cur_slot) {   // a new (b, g) pair: close the previous one, load q
             if (cur_slot >= 0) flush(cur_slot);
             cur_slot = inf.z;
@@ -535,15 +544,16 @@ decode_stream_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict_
                 }
             }
             if (pass == 0) {
-                if (!mbar_wait(&bar[2 * st + 1], ph, abort_flag)) {
+                if (!mbar_wait_warp(&bar[2 * st + 1], ph, abort_flag)) {
                     ok = false;
                     break;
                 }
             }
-            // ---- O += P V for this pass's heads (rows past S_ctx hold stale data: skipped)
+            // ---- O += P V for this pass's heads. Dead keys are skipped, not multiplied by
+            // p = 0: their V rows (masked cache slots, rows past S_ctx) may hold anything.
 #pragma unroll
             for (int kk = 0; kk < kSubKeys; ++kk) {
-                if (kk < rows) {
+                if ((live_bits >> (kk * kBase)) & 1u) {
                     uint32_t wv[C::kEPL / 2];
                     load_bf16_words<C::kEPL>(Vs + kk * C::kRowBytes + lane * C::kEPL * 2, wv);
                     float pk[kHeadsPerPass];
@@ -691,12 +701,65 @@ decode_combine_kernel(Workspace ws, uint16_t* __restrict__ out, int B, int Hkv, 
     }
 }
 
+}  // namespace dec
+}  // namespace attn
+
+#include "decode_mma.cuh"
+
+namespace attn {
+namespace dec {
+
 // ---------------------------------------------------------------- host
+// The stream step runs on the tensor cores (decode_mma.cuh) when num_kv_groups query heads
+// share each K/V byte often enough for the CUDA-core dot products to cost issue slots that
+// compete with the copies; D = 512 keeps the CUDA-core path (its O^T would not fit).
+template <int D, int G>
+constexpr bool use_mma() { return D <= 256 && G >= 4; }
+
+template <int D, int G>
+int launch_stream_mma(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hkv,
+                      int S_ctx, float scale, const Workspace& ws, cudaStream_t stream, int* Pw) {
+    using C = MmaCfg<D>;
+    static std::atomic<int> ctas_for_dev[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -6;
+    int P = ctas_for_dev[dev].load();
+    if (P == 0) {
+        if (cudaFuncSetAttribute(decode_stream_mma_kernel<D, G>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+            cudaSuccess)
+            return -6;
+        int per_sm = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_stream_mma_kernel<D, G>,
+                                                          C::kThreads, C::kSmemBytes) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return -6;
+        P = std::max(1, std::min(Cfg<D>::kMaxWarpsTotal / C::kWarps, per_sm * sms));
+        ctas_for_dev[dev].store(P);
+    }
+    CUtensorMap tk, tv;
+    const uint64_t planes = static_cast<uint64_t>(B) * Hkv;
+    if (encode_map_3d_bf16(&tk, k, D, S_ctx, planes, 64, kSubKeys) ||
+        encode_map_3d_bf16(&tv, v, D, S_ctx, planes, 64, kSubKeys))
+        return -6;
+    *Pw = P * C::kWarps;
+    return launch_pdl(decode_stream_mma_kernel<D, G>, dim3(P), dim3(C::kThreads), C::kSmemBytes,
+                      stream, tk, tv, q, ws, B, Hkv, S_ctx, scale * kLog2e);
+}
+
 template <int D, int G>
 int launch_dg(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* mask,
               uint16_t* out, int B, int Hkv, int S_ctx, float scale, const Workspace& ws,
               cudaStream_t stream) {
     using C = Cfg<D>;
+    if constexpr (use_mma<D, G>()) {
+        if (launch_pdl(decode_scan_kernel, dim3(B), dim3(kScanThreads), 0, stream, mask, S_ctx, ws))
+            return -6;
+        int Pw = 0;
+        if (launch_stream_mma<D, G>(q, k, v, B, Hkv, S_ctx, scale, ws, stream, &Pw)) return -6;
+        return launch_pdl(decode_combine_kernel<D>, dim3(B * Hkv * G), dim3(kCombineThreads), 0,
+                          stream, ws, out, B, Hkv, G, Pw);
+    }
     static std::atomic<int> ctas_for_dev[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -6;

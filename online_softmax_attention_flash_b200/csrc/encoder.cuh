@@ -46,10 +46,11 @@ constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
 // Of every 8 column pairs of an unmasked S tile, this many take 2^x from the FMA-pipe
 // polynomial instead of the MUFU ex2 unit. At D = 64 the exponentials are as many per
-// MMA flop as MUFU can barely sustain, so a share moves to the FMA pipe; at D = 128
-// MUFU has room and the polynomial only costs issue slots.
+// MMA flop as MUFU can barely sustain, so a share moves to the FMA pipe (measured on the
+// ViT-L case: 0/8 35.2 us, 1/8 30.3 us, 2/8 30.6 us per call); at D = 128 the same 1/8
+// share measured 1% faster than none.
 template <int D>
-__host__ __device__ constexpr int poly_eighths() { return D == 64 ? 1 : 0; }
+__host__ __device__ constexpr int poly_eighths() { return 1; }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -166,6 +167,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // set-up done: let the next kernel on the stream start, then wait for the previous one
     pdl_launch_dependents();
     pdl_wait_predecessor();
+    int issued_k = 0, issued_v = 0;   // producer: K / V tiles whose copies were started
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
@@ -176,7 +178,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int p = 0; p < C::kPanels; ++p)
                     tma_load_3d(smem + C::kQOff + t * C::kTileBytes + p * C::kPanelBytes, &tm_q,
                                 bars.q_full, p * 64, row0 + t * kTileM, bh);
-            int issued = 0;
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j % C::kStages;
                 const uint32_t use = j / C::kStages;
@@ -186,23 +187,16 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int p = 0; p < C::kPanels; ++p)
                     tma_load_3d(smem + C::kKOff + st * C::kTileBytes + p * C::kPanelBytes, &tm_k,
                                 &bars.k_full[st], p * 64, j * kTileN, bh);
+                issued_k = j + 1;
                 if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, abort_flag);
-                if (!ok) { issued = j + 1; break; }
+                if (!ok) break;
                 mbar_arrive_expect_tx(&bars.v_full[st], C::kTileBytes);
                 for (int p = 0; p < C::kPanels; ++p)
                     tma_load_3d(smem + C::kVOff + st * C::kTileBytes + p * C::kPanelBytes, &tm_v,
                                 &bars.v_full[st], p * 64, j * kTileN, bh);
-                issued = j + 1;
+                issued_v = j + 1;
             }
-            if (!ok) {
-                // let every copy this thread started land before the CTA exits
-                mbar_wait_drain(bars.q_full, 0);
-                for (int j = (issued > C::kStages ? issued - C::kStages : 0); j < issued; ++j) {
-                    const int st = j % C::kStages;
-                    mbar_wait_drain(&bars.k_full[st], (j / C::kStages) & 1);
-                    mbar_wait_drain(&bars.v_full[st], (j / C::kStages) & 1);
-                }
-            }
+            // on an abort (here or in another role) the copies are drained at teardown
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -323,10 +317,9 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tc_commit(&bars.v_empty[st]);
             }
             }
-            // o_final fires when every MMA above has completed (also on the abort path,
-            // so that TMEM is quiescent before it is freed)
+            // o_final fires when every MMA above has completed (committed on the abort path
+            // too: teardown waits for it before TMEM is freed)
             tc_commit(bars.o_final);
-            if (!ok) mbar_wait_drain(bars.o_final, 0);
         }
         __syncwarp();
     } else {
@@ -354,14 +347,14 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tc_fence_before();   // this warp's TMEM reads of S precede the partner's P writes
             __syncwarp();
             if (lane_id() == 0) mbar_arrive(&bars.xchg[t]);
-            if (!mbar_wait(&bars.xchg[t], phase, abort_flag)) return false;
+            if (!mbar_wait_warp(&bars.xchg[t], phase, abort_flag)) return false;
             tc_fence_after();
             *other = *xslot(buf, hf ^ 1);
             return true;
         };
 
         for (int j = 0; j < n_kv; ++j) {
-            ok = mbar_wait(&bars.s_full[t], j & 1, abort_flag);
+            ok = mbar_wait_warp(&bars.s_full[t], j & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             const int kv0 = j * kTileN;
@@ -386,7 +379,9 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (i >= valid) return -INFINITY;
                 if constexpr (kHasBias) {
                     const float bias = __ldg(kb + i);
-                    return bias == -INFINITY ? -INFINITY : fmaf(sv, scale_log2, bias * kLog2e);
+                    // finite biases stay finite in log2 units (a -FLT_MAX fill keeps its key)
+                    return bias == -INFINITY ? -INFINITY
+                                             : fmaf(sv, scale_log2, fmaxf(bias * kLog2e, -FLT_MAX));
                 } else {
                     return sv * scale_log2;
                 }
@@ -452,7 +447,8 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // previous tile has completed (with P over S, s_full already implied it).
                 if constexpr (C::kSepP) {
                     if (c == 0 && j > 0) {
-                        ok = mbar_wait(&bars.pv_done[t], (j - 1) & 1, abort_flag);
+                        ok = mbar_wait_warp(&bars.pv_done[t], (j - 1) & 1, abort_flag);
+                        if (!ok) break;   // PV_t(j-1) may still read P_t: leave it alone
                         tc_fence_after();
                     }
                 }
@@ -482,7 +478,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // full row sum = both halves
         float l_other = 0.f;
         if (ok) ok = exchange(l_run, n_kv & 1, n_kv & 1, &l_other);
-        if (ok) ok = mbar_wait(bars.o_final, 0, abort_flag);
+        if (ok) ok = mbar_wait_warp(bars.o_final, 0, abort_flag);
         if (ok) {
             tc_fence_after();
             const float l_tot = l_run + l_other;
@@ -505,10 +501,26 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
             }
         }
+        tc_wait_st();   // no TMEM store of this warp is in flight when TMEM is freed
     }
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // Some role gave up (a bounded wait ran out): nothing of this CTA may still be in
+        // flight when it exits. Every copy the producer started lands in shared memory (the
+        // latest fill of each ring stage; earlier fills were consumed before their stage was
+        // refilled), and every MMA completes before TMEM is freed.
+        if (warp == kProducerWarp && lane_id() == 0) {
+            mbar_wait_drain(bars.q_full, 0);
+            for (int j = (issued_k > C::kStages ? issued_k - C::kStages : 0); j < issued_k; ++j)
+                mbar_wait_drain(&bars.k_full[j % C::kStages], (j / C::kStages) & 1);
+            for (int j = (issued_v > C::kStages ? issued_v - C::kStages : 0); j < issued_v; ++j)
+                mbar_wait_drain(&bars.v_full[j % C::kStages], (j / C::kStages) & 1);
+        }
+        if (warp == kMmaWarp && lane_id() == 0) mbar_wait_drain(bars.o_final, 0);
+        __syncwarp();
+    }
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);

@@ -175,6 +175,8 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // keys [0, key_end) are visible to some row of the tile
     const int key_end = causal ? hist + min(row0 + kTileM, q_len) : hist;
     const int n_sub = active ? (key_end + kTileN - 1) / kTileN : 0;
+    bool q_issued = false;            // producer: the Q copy was started
+    int issued_k = 0, issued_v = 0;   // producer: K / V sub-tiles whose copies were started
 
     if (!active) {
         // nothing to compute or store (rows past the sequence, or a bad descriptor)
@@ -187,9 +189,9 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             mbar_arrive_expect_tx(bars.q_full, 4 * kPanel);
             for (int pn = 0; pn < 4; ++pn)
                 tma_load_3d(smem + kStageOff + pn * kPanel, &tm_q, bars.q_full, pn * 64, q0 + row0, h);
+            q_issued = true;
             // the ring doubles as Q staging until the softmax warps have quantised Q
             bool ok = mbar_wait(bars.q_ready, 0, abort_flag);
-            int issued = 0;
             for (int j = 0; j < n_sub && ok; ++j) {
                 const int st = j % kStages;
                 const uint32_t use = j / kStages;
@@ -206,21 +208,16 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tma_load_3d(smem + kKOff + st * kKVTileBytes, &tm_k, &bars.k_full[st], 0, off, c2);
                 tma_load_3d(smem + kKOff + st * kKVTileBytes + kPanel, &tm_k, &bars.k_full[st], 128,
                             off, c2);
+                issued_k = j + 1;
                 if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, abort_flag);
-                if (!ok) { issued = j + 1; break; }
+                if (!ok) break;
                 mbar_arrive_expect_tx(&bars.v_full[st], kKVTileBytes);
                 tma_load_3d(smem + kVOff + st * kKVTileBytes, &tm_v, &bars.v_full[st], 0, off, c2);
                 tma_load_3d(smem + kVOff + st * kKVTileBytes + kPanel, &tm_v, &bars.v_full[st], 128,
                             off, c2);
-                issued = j + 1;
+                issued_v = j + 1;
             }
-            if (!ok) {
-                mbar_wait_drain(bars.q_full, 0);
-                for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-                    mbar_wait_drain(&bars.k_full[j % kStages], (j / kStages) & 1);
-                    mbar_wait_drain(&bars.v_full[j % kStages], (j / kStages) & 1);
-                }
-            }
+            // on an abort (here or in another role) the copies are drained at teardown
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -290,15 +287,14 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc_commit(bars.o_ready);
                 tc_commit(&bars.v_empty[st]);
             }
-            tc_commit(bars.o_final);
-            if (!ok) mbar_wait_drain(bars.o_final, 0);
+            tc_commit(bars.o_final);   // teardown waits for it on an abort
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax warpgroup
         const int r = threadIdx.x;                       // 0..127: query row in the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        bool ok = mbar_wait(bars.q_full, 0, abort_flag);
+        bool ok = mbar_wait_warp(bars.q_full, 0, abort_flag);
         float c_row = 0.f;
         if (ok) {
             // quantise this thread's Q row: x = sq * (hi + lo), sq = amax / 448 (per row)
@@ -368,7 +364,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // this row sees keys [0, lim): the history, plus current tokens up to itself
             const int lim = causal ? hist + row0 + r + 1 : hist;
             const int valid = blk_ok ? max(0, min(kTileN, lim - j * kTileN)) : 0;
-            ok = mbar_wait(&bars.s_full[b], (j >> 1) & 1, abort_flag);
+            ok = mbar_wait_warp(&bars.s_full[b], (j >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             float s[kTileN];
@@ -421,7 +417,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             // O and the P buffer are free once PV of the previous sub-tile has completed
             if (j > 0) {
-                ok = mbar_wait(bars.o_ready, (j - 1) & 1, abort_flag);
+                ok = mbar_wait_warp(bars.o_ready, (j - 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, upd)) {
@@ -441,7 +437,7 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tc_fence_before();
             mbar_arrive(bars.p_ready);
         }
-        if (ok) ok = mbar_wait(bars.o_final, 0, abort_flag);
+        if (ok) ok = mbar_wait_warp(bars.o_final, 0, abort_flag);
         if (ok) {
             tc_fence_after();
             const int row = row0 + r;
@@ -465,10 +461,25 @@ paged_history_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
             }
         }
+        tc_wait_st();   // no TMEM store of this warp is in flight when TMEM is freed
     }
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // Some role gave up (a bounded wait ran out): every copy the producer started lands
+        // (the latest fill of each ring stage; earlier fills were consumed before their
+        // stage was refilled) and every MMA completes before this CTA frees TMEM and exits.
+        if (warp == kProducerWarp && lane_id() == 0) {
+            if (q_issued) mbar_wait_drain(bars.q_full, 0);
+            for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
+                mbar_wait_drain(&bars.k_full[j % kStages], (j / kStages) & 1);
+            for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
+                mbar_wait_drain(&bars.v_full[j % kStages], (j / kStages) & 1);
+        }
+        if (warp == kMmaWarp && lane_id() == 0 && active) mbar_wait_drain(bars.o_final, 0);
+        __syncwarp();
+    }
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);

@@ -6,6 +6,7 @@
 // CTA's own shared memory, one destination per copy.
 #pragma once
 
+#include <cfloat>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -55,8 +56,21 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One poll of phase `parity`. try_wait may suspend the thread for a while before it reports
+// that the phase is still open; builds with ATTN_WAIT_TEST_POLL poll with the non-blocking
+// test_wait instead (the failure-detection tests, whose waits must be able to run out even
+// when the awaited copy is only a little late).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
+#ifdef ATTN_WAIT_TEST_POLL
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -64,12 +78,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
-// Wait limit for every spin in this library: far above any legitimate wait
+// Wait limit for every spin of the compute path: far above any legitimate wait
 // (microseconds), short enough that a stuck kernel returns in about a second.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// ATTN_WAIT_LIMIT_NS may set it at build time (the failure-detection tests build
+// a copy of the library with a limit short enough to run out).
+#ifndef ATTN_WAIT_LIMIT_NS
+#define ATTN_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = ATTN_WAIT_LIMIT_NS;
+// Failed polls between two looks at the clock (a power of two). mbarrier.try_wait may
+// suspend the thread for a while before it reports failure, so the clock is read only
+// now and then; the failure-detection tests look at it after every poll.
+#ifndef ATTN_WAIT_SPINS_PER_CHECK
+#define ATTN_WAIT_SPINS_PER_CHECK 64u
+#endif
+constexpr uint32_t kSpinsPerCheck = ATTN_WAIT_SPINS_PER_CHECK;
+static_assert((kSpinsPerCheck & (kSpinsPerCheck - 1)) == 0, "a power of two");
+// Limit of the teardown drains: always the full second, so that every copy and MMA
+// a CTA has started lands before it exits, whatever kWaitLimitNs is.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 // Bounded wait on phase `parity` of `bar`. Returns false if the wait ran out or
 // if another thread of the CTA already flagged an abort (*abort != 0); in both
@@ -80,7 +111,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     uint32_t spins = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((++spins & 63u) == 0) {
+        if ((++spins & (kSpinsPerCheck - 1)) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 *abort = 1;
@@ -91,11 +122,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait for all 32 lanes of a warp that go on to warp-collective instructions
+// (tcgen05.ld / st, shuffles): the result is the same in every lane (false if any lane's
+// wait failed), so the warp leaves or continues as a whole.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait used only on the teardown path (after an abort): no status update.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+        if (globaltimer_ns() - t0 > kDrainLimitNs) return;
     }
 }
 
@@ -106,6 +145,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
 

@@ -43,6 +43,36 @@ inline int encode_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t e
     return r == CUDA_SUCCESS ? 0 : -6;
 }
 
+// Tiled bf16 maps of rank 2 and 4 (row-major, innermost first), 128-byte swizzle,
+// box0 * 2 = 128 bytes. Out-of-range box elements read as zero.
+inline int encode_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint32_t box0, uint32_t box1) {
+    auto fn = encode_tiled_fn();
+    if (!fn) return -6;
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {d0 * 2};
+    cuuint32_t box[2] = {box0, box1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -6;
+}
+
+inline int encode_map_4d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint64_t d3, uint32_t box0, uint32_t box1) {
+    auto fn = encode_tiled_fn();
+    if (!fn) return -6;
+    cuuint64_t dims[4] = {d0, d1, d2, d3};
+    cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    cuuint32_t box[4] = {box0, box1, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -6;
+}
+
 inline int encode_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                               uint64_t d2, uint32_t box0, uint32_t box1) {
     return encode_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d0, d1, d2, box0, box1);

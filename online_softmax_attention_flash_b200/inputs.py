@@ -208,3 +208,28 @@ def rope_tables(S: int, D: int, base: float = 10000.0):
     w = base ** (-2.0 * j / D)
     theta = torch.arange(S, dtype=torch.float64)[:, None] * w[None, :]
     return torch.cos(theta).float(), torch.sin(theta).float()
+
+
+@dataclass
+class ProjectionCase:
+    x: torch.Tensor            # [B, S, C] bf16 block input
+    w_qkv: torch.Tensor        # [3 H D, C] bf16
+    b_qkv: Optional[torch.Tensor]   # [3 H D] fp32
+    w_o: torch.Tensor          # [C_out, H D] bf16
+    b_o: Optional[torch.Tensor]     # [C_out] fp32
+    H: int
+    D: int
+
+
+def projection_case(B, S, C, H, D, seed, C_out=None, bias=True) -> ProjectionCase:
+    """Random-init weights of a ViT attention block (no trained weights exist here): entries
+    N(0, 1/fan_in) in bf16 like a freshly initialised Linear, biases N(0, 0.02^2) fp32, and a
+    block input x ~ N(0, 1) in bf16 (a LayerNorm output has unit variance per channel)."""
+    g = _gen(seed)
+    C_out = C if C_out is None else C_out
+    x = randn_bf16((B, S, C), g)
+    w_qkv = (torch.randn((3 * H * D, C), generator=g) / C ** 0.5).to(torch.bfloat16)
+    w_o = (torch.randn((C_out, H * D), generator=g) / (H * D) ** 0.5).to(torch.bfloat16)
+    b_qkv = torch.randn(3 * H * D, generator=g) * 0.02 if bias else None
+    b_o = torch.randn(C_out, generator=g) * 0.02 if bias else None
+    return ProjectionCase(x, w_qkv, b_qkv, w_o, b_o, H, D)

@@ -153,3 +153,17 @@ def test_general_finite_key_bias():
     ref = oracle.encoder_attention(to_f64(c.q), to_f64(c.k), to_f64(c.v), c.softmax_scale,
                                    key_bias=kb.double().numpy())
     assert_bf16_parity(out, ref, 2, "general key bias")
+
+
+def test_float32_min_key_bias_keeps_keys():
+    # a finite -FLT_MAX bias keeps its keys: all of them give the mean of V, next to 0-biased
+    # keys they carry no weight (-inf alone removes a key)
+    case = syn.encoder_case(2, 2, 300, 64, seed=94)
+    fmin = torch.finfo(torch.float32).min
+    case.key_bias = torch.zeros(2, 300)
+    case.key_bias[0] = fmin
+    case.key_bias[1, 150:] = fmin
+    got = _run(case)
+    assert_bf16_parity(got, _oracle(case), 2, "finfo.min bias")
+    ref = case.v[0].double().mean(dim=1, keepdim=True).expand(2, 300, 64)
+    assert torch.allclose(got[0].cpu().double(), ref, atol=2e-3, rtol=0)
