@@ -108,3 +108,19 @@ def test_paged_wait_timeout_is_reported(short_wait_lib):
                                          p.k_scale, p.v_scale, p.block_table.numpy(), 512, 3000,
                                          p.softmax_scale, 4)
     assert rel_l2(to_f64(good), ref) <= FP8_REL_L2
+
+
+def test_projection_wait_timeout_is_reported(short_wait_lib):
+    c = syn.projection_case(1, 512, 256, 4, 64, seed=504)
+    x, w, bq = c.x.to(DEV), c.w_qkv.to(DEV), c.b_qkv.to(DEV)
+    q, k, v = (torch.empty((1, 4, 512, 64), dtype=torch.bfloat16, device=DEV) for _ in range(3))
+    seen = _until_timeout(short_wait_lib, lambda: short_wait_lib.attn_qkv_rope_proj(
+        x.data_ptr(), w.data_ptr(), bq.data_ptr(), None, None, 0, 1, 512, 256, 4, 64,
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _stream()))
+    assert seen[-1] == TIMEOUT, seen
+    torch.cuda.synchronize()
+    gq, gk, gv = B.attn_qkv_rope_proj(x, w, bq, 4, 64)
+    assert B.attn_check() == 0
+    ref = oracle.qkv_projection(to_f64(c.x), to_f64(c.w_qkv), c.b_qkv.double().numpy(), 4, 64)
+    for g, r, n in zip((gq, gk, gv), ref, "qkv"):
+        assert_bf16_parity(g, r, 2, f"{n} after a timed-out call")
