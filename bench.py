@@ -202,7 +202,9 @@ class EncoderWork:
         self.launches_per_step = cfg["sets"]
         self.work_per_step = self.flops_per_launch * cfg["sets"]
         self.unit, self.bound = "TFLOP/s", "tensor"
-        self.kernel_regex = "encoder_fwd_kernel"
+        # head dim 64 without a key bias runs the one-query-tile kernel
+        self.kernel_regex = ("encoder_1q_kernel" if D == 64 and self.bias[0] is None
+                             else "encoder_fwd_kernel")
         self.peak_ratio = 1.0
         self.dtype = "bf16"
 
@@ -305,7 +307,10 @@ class DecodeWork:
         self.work_per_step = float(np.mean(self.bytes))
         self.flops_per_launch = self.work_per_step
         self.unit, self.bound = "GB/s", "hbm"
-        self.kernel_regex = "decode_stream_kernel"
+        # 4 or more query heads per kv head (D <= 256) stream on the tensor cores
+        G = cfg["Hq"] // cfg["Hkv"]
+        self.kernel_regex = ("decode_stream_mma_kernel" if G >= 4 and cfg["D"] <= 256
+                             else "decode_stream_kernel")
         self.peak_ratio = 1.0
         self.dtype = "bf16"
         self.i = 0
@@ -450,7 +455,7 @@ class BlockWork:
         self.launches_per_step = 3 * cfg["sets"]
         self.work_per_step = (self.flops_qkv + self.flops_attn + self.flops_out) * cfg["sets"]
         self.unit, self.bound = "TFLOP/s", "tensor"
-        self.kernel_regex = "proj_gemm_kernel|encoder_fwd_kernel"
+        self.kernel_regex = "proj_gemm_kernel|" + ("encoder_1q_kernel" if D == 64 else "encoder_fwd_kernel")
         self.peak_ratio = 1.0
         self.dtype = "bf16"
 

@@ -64,7 +64,9 @@ def _strip_comments(text: str) -> str:
 # shared PTX / tensor-map / status headers and this file's compiler flags).
 KERNEL_SOURCES = {
     "encoder_fwd_kernel": ("encoder.cuh", "attn_lib.cu"),   # launch set-up lives in attn_lib.cu
+    "encoder_1q_kernel": ("encoder1q.cuh", "attn_lib.cu"),
     "decode_stream_kernel": ("decode.cuh",),
+    "decode_stream_mma_kernel": ("decode_mma.cuh", "decode.cuh"),
     "paged_history_kernel": ("paged.cuh",),
     "rope_qk_kernel": ("rope.cuh",),
     "proj_gemm_kernel": ("proj.cuh", "attn_lib.cu"),

@@ -18,6 +18,7 @@
 #include "attn.h"
 #include "decode.cuh"
 #include "encoder.cuh"
+#include "encoder1q.cuh"
 #include "paged.cuh"
 #include "proj.cuh"
 #include "rope.cuh"
@@ -43,6 +44,25 @@ int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
         return ATTN_ERR_CUDA;
     done_mask.fetch_or(bit, std::memory_order_acq_rel);
     return ATTN_OK;
+}
+
+// Head dim 64 without a key bias: one query tile per CTA, two CTAs per SM (encoder1q.cuh).
+int launch_encoder1q(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
+                     int H, int S, float scale, cudaStream_t stream) {
+    using namespace attn::enc1q;
+    static std::atomic<uint64_t> smem_done{0};
+    auto kernel = encoder_1q_kernel;
+    int rc = ensure_smem(kernel, kSmemBytes, smem_done);
+    if (rc) return rc;
+    CUtensorMap tq, tk, tv;
+    const uint64_t rows = static_cast<uint64_t>(S);
+    const uint64_t heads = static_cast<uint64_t>(B) * H;
+    if ((rc = attn::encode_map_3d_bf16(&tq, q, kD, rows, heads, 64, kTileM))) return rc;
+    if ((rc = attn::encode_map_3d_bf16(&tk, k, kD, rows, heads, 64, kTileN))) return rc;
+    if ((rc = attn::encode_map_3d_bf16(&tv, v, kD, rows, heads, 64, kTileN))) return rc;
+    dim3 grid((S + kTileM - 1) / kTileM, static_cast<unsigned>(heads));
+    return attn::launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, out, S,
+                            scale * kLog2e);
 }
 
 template <int D, bool kBias>
@@ -161,7 +181,7 @@ int attn_encoder_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, ui
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (D == 64)
         return key_bias ? launch_encoder<64, true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
-                        : launch_encoder<64, false>(q, k, v, out, B, H, S, softmax_scale, nullptr, st);
+                        : launch_encoder1q(q, k, v, out, B, H, S, softmax_scale, st);
     return key_bias ? launch_encoder<128, true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
                     : launch_encoder<128, false>(q, k, v, out, B, H, S, softmax_scale, nullptr, st);
 }

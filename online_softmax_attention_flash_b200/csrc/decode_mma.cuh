@@ -147,7 +147,7 @@ decode_stream_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     fill_window();
     int next_x = 0;                 // first item of the next step to issue
     int issued_k = 0, issued_v = 0; // steps whose K / V copies were started
-    int pend_bg = 0, pend_k0[2] = {0, 0}, pend_n = 0;   // V half still to be issued (lane 0)
+    int pend_bg = 0, pend_k0a = 0, pend_k0b = 0, pend_n = 0;   // V half still to be issued (lane 0)
     constexpr uint32_t kItemBytes = C::kPanels * 1024;   // one 8-key box per panel
     // Issue the K half (and the mask) of step `t` starting at item next_x; whole warp calls.
     auto issue_k = [&](int t) {
@@ -172,8 +172,8 @@ decode_stream_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             uint8_t* kdst = ring_p + st * C::kStageBytes;
             info[st] = make_int4(cnt, slot0, bg0, 0);
             pend_bg = bg0;
-            pend_k0[0] = sub0 * kSubKeys;
-            pend_k0[1] = sub1 * kSubKeys;
+            pend_k0a = sub0 * kSubKeys;
+            pend_k0b = sub1 * kSubKeys;
             pend_n = cnt;
             mbar_arrive_expect_tx(&bar[2 * st], cnt * (kItemBytes + kSubKeys * 4));
             for (int it = 0; it < cnt; ++it) {
@@ -181,7 +181,7 @@ decode_stream_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                           kSubKeys * 4, &bar[2 * st]);
                 for (int p = 0; p < C::kPanels; ++p)
                     tma_load_3d(kdst + p * C::kPanelBytes + it * 1024, &tm_k, &bar[2 * st], p * 64,
-                                pend_k0[it], bg0);
+                                it ? pend_k0b : pend_k0a, bg0);
             }
             issued_k = t + 1;
         }
@@ -194,7 +194,7 @@ decode_stream_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         for (int it = 0; it < pend_n; ++it)
             for (int p = 0; p < C::kPanels; ++p)
                 tma_load_3d(vdst + p * C::kPanelBytes + it * 1024, &tm_v, &bar[2 * st + 1], p * 64,
-                            pend_k0[it], pend_bg);
+                            it ? pend_k0b : pend_k0a, pend_bg);
         issued_v = t + 1;
     };
     int n_steps_issued = 0;

@@ -361,53 +361,74 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int valid = S - kv0;   // keys of this tile that exist
             const float* kb = nullptr;
             bool full_tile = !kHasBias && valid >= kTileN;
+            bool bias_zero = true;
             if constexpr (kHasBias) {
                 kb = key_bias + static_cast<size_t>(b) * S + kv0;
-                // A complete tile whose 64 bias values of this warp's half are all zero is
-                // computed exactly as without a bias (the common case of right padding: only
+                // A tile whose bias values (of this warp's half, columns before S) are all zero
+                // is computed exactly as without a bias (the common case of right padding: only
                 // the tiles past a sequence's length carry -inf).
-                bool zero = valid >= kTileN;
-                if (zero) {
-                    const int c = col0 + 2 * static_cast<int>(lane_id());
-                    zero = __ldg(kb + c) == 0.f && __ldg(kb + c + 1) == 0.f;
-                }
-                full_tile = __all_sync(0xffffffffu, zero);
+                const int c = col0 + 2 * static_cast<int>(lane_id());
+                const bool zero = (c >= valid || __ldg(kb + c) == 0.f) &&
+                                  (c + 1 >= valid || __ldg(kb + c + 1) == 0.f);
+                bias_zero = __all_sync(0xffffffffu, zero);
+                full_tile = bias_zero && valid >= kTileN;
             }
-            // score of tile column i in log2 units (scale folded in), -inf where masked;
-            // only used on masked tiles (bias or a ragged last tile)
-            auto masked_score = [&](float sv, int i) -> float {
-                if (i >= valid) return -INFINITY;
-                if constexpr (kHasBias) {
-                    const float bias = __ldg(kb + i);
-                    // finite biases stay finite in log2 units (a -FLT_MAX fill keeps its key)
-                    return bias == -INFINITY ? -INFINITY
-                                             : fmaf(sv, scale_log2, fmaxf(bias * kLog2e, -FLT_MAX));
-                } else {
-                    return sv * scale_log2;
-                }
-            };
             uint32_t u[kHalf];
             tmem_ld64_wait(tSh, u);
+            // A ragged last tile without a key bias keeps the raw-score path: the columns
+            // past S become -inf (the scale is positive, so the max is unchanged and every
+            // exponential of them is exactly 0); only MUFU exponentials are used there.
+            const bool raw_path = !kHasBias || bias_zero;
+            if (raw_path && valid < kTileN) {
+#pragma unroll
+                for (int i = 0; i < kHalf; ++i)
+                    if (col0 + i >= valid) u[i] = __float_as_uint(-INFINITY);
+            }
             if constexpr (C::kSepP) {   // S_t may be overwritten by the next QK from here on
                 tc_fence_before();
                 __syncwarp();
                 if (lane_id() == 0) mbar_arrive(&bars.s_free[t]);
             }
             float m_half;
-            if (full_tile) {
-                float mx[4] = {__uint_as_float(u[0]), __uint_as_float(u[1]), __uint_as_float(u[2]),
-                               __uint_as_float(u[3])};
+            if (raw_path) {
+                // pairs first, then three-input maxes over groups of 8 columns
+                static_assert(kHalf % 8 == 0, "row max reads whole groups of 8 columns");
+                float mx[4];
 #pragma unroll
-                for (int i = 4; i < kHalf; i += 8) {
+                for (int e = 0; e < 4; ++e)
+                    mx[e] = fmaxf(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+#pragma unroll
+                for (int i = 8; i < kHalf; i += 8) {
                     mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
                     mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
                     mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
                     mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
                 }
                 m_half = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
-            } else {
+            } else if constexpr (kHasBias) {
+                // key bias on this tile: score of column i in log2 units (scale folded in),
+                // -inf where masked; finite biases stay finite (a -FLT_MAX fill keeps its key).
+                // Every lane reads the same biases: 16-byte broadcast loads, 4 columns each.
 #pragma unroll
-                for (int i = 0; i < kHalf; ++i) u[i] = __float_as_uint(masked_score(__uint_as_float(u[i]), col0 + i));
+                for (int i = 0; i < kHalf; i += 4) {
+                    float4 b4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                    if (col0 + i + 3 < valid && ((reinterpret_cast<uintptr_t>(kb + col0 + i) & 15u) == 0)) {
+                        b4 = __ldg(reinterpret_cast<const float4*>(kb + col0 + i));
+                    } else {
+                        if (col0 + i < valid) b4.x = __ldg(kb + col0 + i);
+                        if (col0 + i + 1 < valid) b4.y = __ldg(kb + col0 + i + 1);
+                        if (col0 + i + 2 < valid) b4.z = __ldg(kb + col0 + i + 2);
+                        if (col0 + i + 3 < valid) b4.w = __ldg(kb + col0 + i + 3);
+                    }
+                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float sv = __uint_as_float(u[i + e]);
+                        u[i + e] = __float_as_uint(bb[e] == -INFINITY
+                                                       ? -INFINITY
+                                                       : fmaf(sv, scale_log2, fmaxf(bb[e] * kLog2e, -FLT_MAX)));
+                    }
+                }
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(u[i]));
@@ -431,10 +452,10 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const int kk = c * 16 + k;   // column pair index in this half
                     const float2 sv = make_float2(__uint_as_float(u[2 * kk]), __uint_as_float(u[2 * kk + 1]));
                     float2 pv;
-                    if (full_tile) {
+                    if (raw_path) {
                         const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
                                                     make_float2(-m_use, -m_use));
-                        if ((kk & 7) < poly_eighths<D>()) pv = exp2_poly2(x);
+                        if (full_tile && (kk & 7) < poly_eighths<D>()) pv = exp2_poly2(x);
                         else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     } else {
                         pv = make_float2(ex2_approx(sv.x - m_use), ex2_approx(sv.y - m_use));

@@ -1,0 +1,319 @@
+// encoder1q.cuh -- non-causal encoder attention forward at head_dim 64, one query tile per
+// CTA, two CTAs per SM (sm_100a).
+//
+// What it computes: the same as encoder_fwd_kernel (encoder.cuh) for D = 64 without a key
+// bias: out[b,h] = softmax(scale * Q K^T) V, q/k/v/out [B, H, S, 64] bf16. (With a key bias
+// the two-tile kernel runs: a bias on 128 columns per thread costs registers this kernel,
+// at two CTAs per SM, does not have.)
+//
+// How. A CTA owns 128 query rows of one (b, h) and streams the key sequence in 128-key
+// tiles through a 2-stage TMA ring: warp 5 (one thread) issues QK(j+1) as soon as the
+// softmax has read S(j) and PV(j) once P(j) is written; warps 0-3 are the softmax, one
+// thread per row holding all 128 scores of its row, so the row max needs no exchange
+// between warps. TMEM holds S (128 columns), O (64) and P (64, bf16 pairs): 256 columns,
+// and the CTA needs ~81 KB of shared memory, so two CTAs share an SM. The two query tiles
+// an SM works on then belong to different CTAs: nothing in the issue order couples their
+// phases, and one CTA's exponentials (MUFU) overlap the other's max, stores and waits.
+// The running max may be stale by up to 2^8 (the final O / l uses the same reference);
+// two column pairs in eight take 2^x from the FMA-pipe polynomial.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace attn {
+namespace enc1q {
+
+constexpr int kTileM = 128;
+constexpr int kTileN = 128;
+constexpr int kD = 64;
+constexpr int kThreads = 192;          // warps 0-3 softmax, 4 producer, 5 MMA issuer
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kStages = 2;
+constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColO = 128, kColP = 192;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPolyEighths = 2;
+
+constexpr int kQOff = 0;
+constexpr int kKOff = kQOff + kTileBytes;
+constexpr int kVOff = kKOff + kStages * kTileBytes;
+constexpr int kBarOff = kVOff + kStages * kTileBytes;
+// q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full, s_free, p_ready, pv_done,
+// o_final, mma_done
+constexpr int kNumBars = 1 + 4 * kStages + 6;
+constexpr int kMiscOff = kBarOff + kNumBars * 8;
+constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+
+__global__ void __launch_bounds__(kThreads, 2)
+encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int S,
+                  float scale_log2) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + kBarOff);
+    uint64_t* k_full = q_full + 1;
+    uint64_t* k_empty = k_full + kStages;
+    uint64_t* v_full = k_empty + kStages;
+    uint64_t* v_empty = v_full + kStages;
+    uint64_t* s_full = v_empty + kStages;
+    uint64_t* s_free = s_full + 1;
+    uint64_t* p_ready = s_free + 1;
+    uint64_t* pv_done = p_ready + 1;
+    uint64_t* o_final = pv_done + 1;
+    uint64_t* mma_done = o_final + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int bh = blockIdx.y;
+    const int row0 = blockIdx.x * kTileM;
+    const int n_kv = (S + kTileN - 1) / kTileN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);    // one arrival per softmax warp
+        mbar_init(p_ready, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(o_final, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane_id() == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+    pdl_wait_predecessor();
+    int issued_k = 0, issued_v = 0;
+
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane_id() == 0) {
+            bool ok = true;
+            mbar_arrive_expect_tx(q_full, kTileBytes);
+            tma_load_3d(smem + kQOff, &tm_q, q_full, 0, row0, bh);
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int st = j % kStages;
+                const uint32_t use = j / kStages;
+                if (use > 0) ok = mbar_wait(&k_empty[st], (use - 1) & 1, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+                tma_load_3d(smem + kKOff + st * kTileBytes, &tm_k, &k_full[st], 0, j * kTileN, bh);
+                issued_k = j + 1;
+                if (use > 0) ok = mbar_wait(&v_empty[st], (use - 1) & 1, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+                tma_load_3d(smem + kVOff + st * kTileBytes, &tm_v, &v_full[st], 0, j * kTileN, bh);
+                issued_v = j + 1;
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane_id() == 0) {
+            constexpr uint32_t idesc_qk = make_idesc(kTileM, kTileN, 1, 1, 0, 0);
+            constexpr uint32_t idesc_pv = make_idesc(kTileM, kD, 1, 1, 0, 1);
+            const uint64_t dq = smem_desc(smem_u32(smem + kQOff), 16, 1024);
+            const uint64_t dk = smem_desc(smem_u32(smem + kKOff), 16, 1024);
+            const uint64_t dv = smem_desc(smem_u32(smem + kVOff), kTileBytes, 1024);
+            auto issue_qk = [&](int st) {
+                const uint64_t ka = dk + static_cast<uint64_t>((st * kTileBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_f16_ss(tmem_base + kColS, dq + 2 * kk, ka + 2 * kk, idesc_qk, kk > 0);
+            };
+            auto issue_pv = [&](int st, bool acc) {
+                const uint64_t va = dv + static_cast<uint64_t>((st * kTileBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk)
+                    mma_f16_ts(tmem_base + kColO, tmem_base + kColP + kk * 8,
+                               va + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
+                               (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_qk(0);
+                tc_commit(s_full);
+                tc_commit(&k_empty[0]);
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                if (j + 1 < n_kv) {   // S(j+1) once the softmax has read S(j)
+                    const int stn = (j + 1) % kStages;
+                    ok = mbar_wait(s_free, j & 1, abort_flag) &&
+                         mbar_wait(&k_full[stn], ((j + 1) / kStages) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(stn);
+                    tc_commit(s_full);
+                    tc_commit(&k_empty[stn]);
+                }
+                const int st = j % kStages;
+                ok = mbar_wait(p_ready, j & 1, abort_flag) &&
+                     mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(st, j > 0);
+                tc_commit(pv_done);
+                tc_commit(&v_empty[st]);
+            }
+            if (ok) tc_commit(o_final);
+            tc_commit(mma_done);   // teardown waits for it on an abort
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax: one thread per row
+        const int r = threadIdx.x;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tS = tmem_base + lane_off + kColS;
+        const uint32_t tO = tmem_base + lane_off + kColO;
+        const uint32_t tP = tmem_base + lane_off + kColP;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            ok = mbar_wait_warp(s_full, j & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const int kv0 = j * kTileN;
+            const int valid = S - kv0;
+            uint32_t u[kTileN];
+            tmem_ld128_wait(tS, u);
+            tc_fence_before();     // S may be overwritten by QK(j+1) from here on
+            __syncwarp();
+            if (lane_id() == 0) mbar_arrive(s_free);
+            // raw scores (scale folded into the exponent); columns past S are -inf
+            const bool full_tile = valid >= kTileN;
+            if (!full_tile) {
+#pragma unroll
+                for (int i = 0; i < kTileN; ++i)
+                    if (i >= valid) u[i] = __float_as_uint(-INFINITY);
+            }
+            // pairs first, then three-input maxes over groups of 8 columns
+            static_assert(kTileN % 8 == 0, "row max reads whole groups of 8 columns");
+            float mx[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                mx[e] = fmaxf(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+#pragma unroll
+            for (int i = 8; i < kTileN; i += 8) {
+                mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+                mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
+                mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
+                mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
+            }
+            const float m_tile = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
+            const bool upd = m_tile > m_run + kRescaleThreshold;
+            const float m_next = upd ? m_tile : m_run;
+            const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
+            const float alpha = upd ? ex2_approx(m_run - m_use) : 1.f;
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < kTileN / 32; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int kk = c * 16 + k;   // column pair index
+                    const float2 sv = make_float2(__uint_as_float(u[2 * kk]), __uint_as_float(u[2 * kk + 1]));
+                    const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
+                                                make_float2(-m_use, -m_use));
+                    float2 pv;
+                    if (full_tile && (kk & 7) < kPolyEighths) pv = exp2_poly2(x);
+                    else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    if (k & 1) acc1 = __fadd2_rn(acc1, pv);
+                    else acc0 = __fadd2_rn(acc0, pv);
+                    pk[k] = pack_bf16x2(pv.x, pv.y);
+                }
+                // P and O are free once PV of the previous tile has completed
+                if (c == 0 && j > 0) {
+                    ok = mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                tmem_st16(tP + c * 16, pk);
+            }
+            if (!ok) break;
+            l_run = l_run * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+            m_run = m_next;
+            if (j > 0 && __any_sync(0xffffffffu, upd)) {
+#pragma unroll
+                for (int c = 0; c < kD / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32_wait(tO + c * 32, w);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                    tmem_st32(tO + c * 32, w);
+                }
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane_id() == 0) mbar_arrive(p_ready);
+        }
+        if (ok) ok = mbar_wait_warp(o_final, 0, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            const int row = row0 + r;
+            const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+            uint16_t* orow = out + (static_cast<size_t>(bh) * S + row) * kD;
+#pragma unroll
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t w[32];
+                tmem_ld32_wait(tO + c * 32, w);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(w[2 * i]) * inv_l, __uint_as_float(w[2 * i + 1]) * inv_l);
+                if (row < S) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+        }
+        tc_wait_st();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        // a bounded wait ran out: every started copy lands and every MMA completes before
+        // TMEM is freed and the CTA exits
+        if (warp == kProducerWarp && lane_id() == 0) {
+            mbar_wait_drain(q_full, 0);
+            for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
+                mbar_wait_drain(&k_full[j % kStages], (j / kStages) & 1);
+            for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
+                mbar_wait_drain(&v_full[j % kStages], (j / kStages) & 1);
+        }
+        if (warp == kMmaWarp && lane_id() == 0) mbar_wait_drain(mma_done, 0);
+        __syncwarp();
+    }
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace enc1q
+}  // namespace attn

@@ -7,7 +7,7 @@ import torch
 import oracle
 from online_softmax_attention_flash_b200 import binding as B
 from online_softmax_attention_flash_b200 import inputs as syn
-from parity import assert_bf16_parity, to_f64
+from parity import assert_bf16_parity, rel_l2, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -128,16 +128,32 @@ def test_gte_shapes_right_padded_batches(L):
     assert_bf16_parity(out, ref, 2, f"gte L={L}")
 
 
-@pytest.mark.parametrize("D", [64, 128])
-def test_all_zero_key_bias_equals_no_bias_bitwise(D):
-    """Tiles whose key bias is all zero take the unbiased path: identical results."""
-    c = syn.encoder_case(2, 4, 700, D, seed=77, softmax_scale=D ** -0.5)
+def test_all_zero_key_bias_equals_no_bias_bitwise():
+    """Tiles whose key bias is all zero take the unbiased path of the same kernel: identical
+    results (head dim 128, where both calls run the two-tile kernel)."""
+    c = syn.encoder_case(2, 4, 700, 128, seed=77, softmax_scale=128 ** -0.5)
     q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
     zero = torch.zeros((2, 700), dtype=torch.float32, device=DEV)
     a = B.attn_encoder_fwd(q, k, v, c.softmax_scale)
     b = B.attn_encoder_fwd(q, k, v, c.softmax_scale, key_bias=zero)
     assert B.attn_check() == 0
     assert torch.equal(a, b)
+
+
+def test_all_zero_key_bias_d64_agrees_with_no_bias():
+    """Head dim 64: without a bias the one-query-tile kernel runs, with an all-zero bias the
+    two-tile kernel's unbiased path. Both follow the oracle, and they agree closely (the
+    polynomial takes different column pairs, so not bit for bit)."""
+    c = syn.encoder_case(2, 4, 700, 64, seed=77, softmax_scale=0.125)
+    q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
+    zero = torch.zeros((2, 700), dtype=torch.float32, device=DEV)
+    a = B.attn_encoder_fwd(q, k, v, c.softmax_scale)
+    b = B.attn_encoder_fwd(q, k, v, c.softmax_scale, key_bias=zero)
+    assert B.attn_check() == 0
+    ref = _oracle(c)
+    assert_bf16_parity(a, ref, 2, "no bias")
+    assert_bf16_parity(b, ref, 2, "all-zero bias")
+    assert rel_l2(to_f64(a), to_f64(b)) <= 2e-3
 
 
 def test_general_finite_key_bias():
@@ -167,3 +183,23 @@ def test_float32_min_key_bias_keeps_keys():
     assert_bf16_parity(got, _oracle(case), 2, "finfo.min bias")
     ref = case.v[0].double().mean(dim=1, keepdim=True).expand(2, 300, 64)
     assert torch.allclose(got[0].cpu().double(), ref, atol=2e-3, rtol=0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S", [300, 512])
+def test_all_scores_far_below_zero(D, S):
+    """Every score of every row near -1600 in natural units: the row max must be taken over
+    exactly the row's scores (any stray larger value makes every weight underflow to 0)."""
+    c = syn.encoder_case(1, 2, S, D, seed=95, softmax_scale=D ** -0.5)
+    g = torch.Generator().manual_seed(96)
+    k0 = torch.randn(D, generator=g)
+    k0 = k0 / k0.norm() * D ** 0.25 * 8.0            # |k0|^2 * scale = 64
+    kk = k0 + 0.05 * torch.randn((1, 2, S, D), generator=g)
+    c.k = kk.to(torch.bfloat16)
+    c.q = (-25.0 * k0).expand(1, 2, S, D).to(torch.bfloat16).contiguous()
+    got = _run(c)
+    ref = _oracle(c)
+    s_max = (to_f64(c.q)[0, 0, 0] @ to_f64(c.k)[0, 0].T).max() * c.softmax_scale
+    assert s_max < -1000.0, s_max                     # the case is what it claims
+    assert_bf16_parity(got, ref, 2, "scores far below zero")
+

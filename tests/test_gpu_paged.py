@@ -7,7 +7,7 @@ import torch
 import oracle
 from online_softmax_attention_flash_b200 import binding as B
 from online_softmax_attention_flash_b200 import inputs as syn
-from parity import FP8_REL_L2, head_cosines, rel_l2, to_f64
+from parity import FP8_REL_L2, FP8_ROW_REL_L2, assert_rows_close, head_cosines, rel_l2, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +40,7 @@ def _check(got_t, ref, what, bound=FP8_REL_L2):
     e = rel_l2(got, ref)
     assert e <= FP8_REL_L2, f"{what}: rel_l2 {e:.3e}"
     assert e <= bound, f"{what}: rel_l2 {e:.3e} above the split-e4m3 design bound {bound}"
+    assert_rows_close(got, ref, FP8_ROW_REL_L2, what)
     return e
 
 

@@ -58,19 +58,25 @@ def _until_timeout(lib, launch, tries=5):
     return seen
 
 
-def test_encoder_wait_timeout_is_reported(short_wait_lib):
-    c = syn.encoder_case(1, 4, 1024, 64, seed=501)
+@pytest.mark.parametrize("D,with_bias", [(64, False), (64, True), (128, False)],
+                         ids=["d64_one_tile", "d64_key_bias_two_tile", "d128_two_tile"])
+def test_encoder_wait_timeout_is_reported(short_wait_lib, D, with_bias):
+    c = syn.encoder_case(1, 4, 1024, D, seed=501)
     q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
+    kb = torch.zeros((1, 1024), dtype=torch.float32, device=DEV) if with_bias else None
+    if kb is not None:
+        kb[0, 900:] = float("-inf")
     out = torch.empty_like(q)
     seen = _until_timeout(short_wait_lib, lambda: short_wait_lib.attn_encoder_fwd(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), 1, 4, 1024, 64, 0.125, None,
-        _stream()))
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), 1, 4, 1024, D, 0.125,
+        None if kb is None else kb.data_ptr(), _stream()))
     assert seen[-1] == TIMEOUT, seen
     torch.cuda.synchronize()   # the context is intact
     # the product library, same process, same inputs: exact as ever
-    good = B.attn_encoder_fwd(q, k, v, 0.125)
+    good = B.attn_encoder_fwd(q, k, v, 0.125, key_bias=kb)
     assert B.attn_check() == 0
-    ref = oracle.encoder_attention(to_f64(c.q), to_f64(c.k), to_f64(c.v), 0.125)
+    ref = oracle.encoder_attention(to_f64(c.q), to_f64(c.k), to_f64(c.v), 0.125,
+                                   key_bias=None if kb is None else kb.double().cpu().numpy())
     assert_bf16_parity(good, ref, 2, "encoder after a timed-out call")
 
 
