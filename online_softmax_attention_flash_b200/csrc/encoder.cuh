@@ -360,7 +360,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int kv0 = j * kTileN;
             const int valid = S - kv0;   // keys of this tile that exist
             const float* kb = nullptr;
-            bool full_tile = !kHasBias && valid >= kTileN;
             bool bias_zero = true;
             if constexpr (kHasBias) {
                 kb = key_bias + static_cast<size_t>(b) * S + kv0;
@@ -371,13 +370,13 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const bool zero = (c >= valid || __ldg(kb + c) == 0.f) &&
                                   (c + 1 >= valid || __ldg(kb + c + 1) == 0.f);
                 bias_zero = __all_sync(0xffffffffu, zero);
-                full_tile = bias_zero && valid >= kTileN;
             }
             uint32_t u[kHalf];
             tmem_ld64_wait(tSh, u);
             // A ragged last tile without a key bias keeps the raw-score path: the columns
-            // past S become -inf (the scale is positive, so the max is unchanged and every
-            // exponential of them is exactly 0); only MUFU exponentials are used there.
+            // past S become -inf (the scale is positive, so the max is unchanged); their
+            // weights are 0, or 2^-125 where the polynomial takes them, against V rows that
+            // the copy zero-filled.
             const bool raw_path = !kHasBias || bias_zero;
             if (raw_path && valid < kTileN) {
 #pragma unroll
@@ -455,7 +454,9 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (raw_path) {
                         const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
                                                     make_float2(-m_use, -m_use));
-                        if (full_tile && (kk & 7) < poly_eighths<D>()) pv = exp2_poly2(x);
+                        // the polynomial also takes the -inf columns past S of a ragged tile:
+                        // it clamps them to 2^-125, and their V rows are zero-filled
+                        if ((kk & 7) < poly_eighths<D>()) pv = exp2_poly2(x);
                         else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     } else {
                         pv = make_float2(ex2_approx(sv.x - m_use), ex2_approx(sv.y - m_use));

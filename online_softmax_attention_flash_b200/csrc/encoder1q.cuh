@@ -190,9 +190,12 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t tP = tmem_base + lane_off + kColP;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
+        bool s_seen = false;   // S(j) already reported complete by an earlier look
         for (int j = 0; j < n_kv; ++j) {
-            ok = mbar_wait_warp(s_full, j & 1, abort_flag);
-            if (!ok) break;
+            if (!__all_sync(0xffffffffu, s_seen)) {
+                ok = mbar_wait_warp(s_full, j & 1, abort_flag);
+                if (!ok) break;
+            }
             tc_fence_after();
             const int kv0 = j * kTileN;
             const int valid = S - kv0;
@@ -201,9 +204,11 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_before();     // S may be overwritten by QK(j+1) from here on
             __syncwarp();
             if (lane_id() == 0) mbar_arrive(s_free);
+            // PV(j-1) was issued when P(j-1) was complete and has most likely finished: look
+            // now, use the answer before P(j) is stored
+            const bool pv_seen = j == 0 || mbar_test(pv_done, (j - 1) & 1);
             // raw scores (scale folded into the exponent); columns past S are -inf
-            const bool full_tile = valid >= kTileN;
-            if (!full_tile) {
+            if (valid < kTileN) {
 #pragma unroll
                 for (int i = 0; i < kTileN; ++i)
                     if (i >= valid) u[i] = __float_as_uint(-INFINITY);
@@ -237,7 +242,10 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
                                                 make_float2(-m_use, -m_use));
                     float2 pv;
-                    if (full_tile && (kk & 7) < kPolyEighths) pv = exp2_poly2(x);
+                    // the polynomial also takes the -inf columns of a ragged tile: it clamps
+                    // them to 2^-125, and as past S the V rows are zero-filled they add
+                    // nothing to O (and less than an ulp to the row sum)
+                    if ((kk & 7) < kPolyEighths) pv = exp2_poly2(x);
                     else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     if (k & 1) acc1 = __fadd2_rn(acc1, pv);
                     else acc0 = __fadd2_rn(acc0, pv);
@@ -245,10 +253,14 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 // P and O are free once PV of the previous tile has completed
                 if (c == 0 && j > 0) {
-                    ok = mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag);
-                    if (!ok) break;
+                    if (!__all_sync(0xffffffffu, pv_seen)) {
+                        ok = mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag);
+                        if (!ok) break;
+                    }
                     tc_fence_after();
                 }
+                // QK(j+1) was issued when S(j) had been read: look now whether S(j+1) is in
+                if (c == kTileN / 32 - 1) s_seen = j + 1 < n_kv && mbar_test(s_full, (j + 1) & 1);
                 tmem_st16(tP + c * 16, pk);
             }
             if (!ok) break;

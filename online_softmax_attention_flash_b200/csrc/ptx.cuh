@@ -82,6 +82,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking look at phase `parity` (acquire when it reports completion): issued early, its
+// answer can be consumed later, so that a phase already complete costs no wait.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait limit for every spin of the compute path: far above any legitimate wait
 // (microseconds), short enough that a stuck kernel returns in about a second.
 // ATTN_WAIT_LIMIT_NS may set it at build time (the failure-detection tests build
