@@ -862,8 +862,9 @@ def time_work(work, workload, steps, warmup, info, device, stream, use_graph):
 def roofline_of(work, workload, total_ms, steps, clocks=None):
     """Dominant kernel: algorithmic work per launch / mean launch time against the peak.
     Tensor-bound kernels are held against the burst GEMM peak when timed alone, and against
-    the sustained one when the timed region is long (over a second) or the clocks show that
-    the 1 kW power cap was holding the GPU back meanwhile."""
+    the sustained one when the timed region is long (over a second) or the 1 kW power cap
+    held the SM clock down meanwhile (sw_power_cap active and a median clock more than 5%
+    below the maximum; a cap that leaves the clock at its maximum changes nothing)."""
     peaks, peak_src = load_peaks()
     per_launch_ms = total_ms / (steps * work.launches_per_step)
     if work.bound == "hbm":
@@ -874,7 +875,9 @@ def roofline_of(work, workload, total_ms, steps, clocks=None):
         peak_name = "hbm_gbs"
     else:
         achieved = work.flops_per_launch / (per_launch_ms / 1e3) / 1e12
-        capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+        capped = (bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+                  and clocks.get("sm_mhz") is not None and clocks.get("sm_max_mhz")
+                  and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
         sustained = total_ms > 1000.0 or capped
         peak_name = "bf16_tflops_sustained" if sustained else "bf16_tflops"
         peak = float(peaks[peak_name]) * work.peak_ratio

@@ -53,6 +53,7 @@ def test_qkv_rope_vitl_layer(mode):
     (1, 300, 256, 4, 128, "interleaved", True),   # D = 128
     (3, 129, 192, 6, 64, None, True),             # no rotation, 3 batch entries
     (1, 1, 64, 2, 64, "half", True),              # a single token
+    (2, 600, 256, 4, 64, "half", True),           # 256-token tiles, ragged third tile
 ])
 def test_qkv_shapes(B_, S, C, H, D, mode, bias):
     case = syn.projection_case(B_, S, C, H, D, seed=3200 + S + D, bias=bias)
@@ -62,9 +63,10 @@ def test_qkv_shapes(B_, S, C, H, D, mode, bias):
         assert_bf16_parity(g, r, 2, f"{n} S={S} D={D} {mode}")
 
 
-def test_qkv_one_hot_weights_are_bit_exact():
+@pytest.mark.parametrize("S,H", [(150, 2), (300, 4)])   # 128- and 256-token tiles
+def test_qkv_one_hot_weights_are_bit_exact(S, H):
     # W = three stacked identities (C = H D): q = k = v = x laid out as heads, bit for bit
-    Bn, S, H, D = 2, 150, 2, 64
+    Bn, D = 2, 64
     C = H * D
     x = syn.randn_bf16((Bn, S, C), torch.Generator().manual_seed(3300))
     w = torch.cat([torch.eye(C)] * 3).to(torch.bfloat16)
