@@ -72,7 +72,11 @@ typedef enum attn_status {
  *   softmax_scale: finite, > 0 (1/sqrt(D) for the ViT encoders).
  *   key_bias     : NULL, or [B, S] fp32 additive bias added to every query's
  *                  score for key j of batch entry b (0 keep, -inf drop; any
- *                  finite value, -FLT_MAX included, keeps the key).
+ *                  finite value, -FLT_MAX included, keeps the key). The 128-key
+ *                  tiles after the last kept key of an entry are never read (so
+ *                  their K and V may hold anything); a dropped key inside a tile
+ *                  that holds a kept key has weight 0, but its V row is still
+ *                  multiplied by it and must be finite.
  *
  * Every query row attends to all S keys (no causal mask). Accumulation is fp32;
  * out is rounded to bf16 (round-to-nearest-even).

@@ -67,8 +67,9 @@ struct Cfg {
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
     // o_final, xchg[2] (row-max / row-sum exchange between the two halves of a tile),
-    // s_free[2] (softmax has read S_t), pv_done[2] (PV_t has completed)
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 2 + 2;
+    // s_free[2] (softmax has read S_t), pv_done[2] (PV_t has completed), count_ready (the
+    // number of key tiles with a kept key is known; key-bias kernels)
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 2 + 2 + 1;
     static constexpr int kXchgOff = kBarOff + kNumBars * 8;   // float [2 buf][2 tile][2 half][128]
     static constexpr int kMiscOff = kXchgOff + 2 * 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + tmem slot, abort flag, alignment slack
@@ -94,6 +95,7 @@ struct Bars {
     uint64_t* xchg;
     uint64_t* s_free;
     uint64_t* pv_done;
+    uint64_t* count_ready;
 };
 
 template <int D>
@@ -112,7 +114,19 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
     r.xchg = r.o_final + 1;
     r.s_free = r.xchg + 2;
     r.pv_done = r.s_free + 2;
+    r.count_ready = r.pv_done + 2;
     return r;
+}
+
+// Key tiles up to the last key whose bias is not -inf (at least one), found by a whole warp:
+// with right padding the trailing tiles hold only -inf keys, which take no part in any row.
+__device__ __forceinline__ int live_key_tiles(const float* kb, int S) {
+    int last = -1;
+    for (int c = static_cast<int>(lane_id()); c < S; c += 32)
+        if (__ldg(kb + c) != -INFINITY) last = c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    return max(1, (last + kTileN) / kTileN);
 }
 
 template <int D, bool kHasBias>
@@ -130,7 +144,10 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int warp = threadIdx.x >> 5;
     const int bh = blockIdx.y;
     const int row0 = blockIdx.x * kRowsPerCta;
-    const int n_kv = (S + kTileN - 1) / kTileN;
+    const int n_kv_all = (S + kTileN - 1) / kTileN;
+    // with a key bias: the key tiles that hold a kept key (the producer counts them while the
+    // first copies are in flight and publishes the count here)
+    volatile int* n_live_slot = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
 
     if (threadIdx.x == 0) {
         mbar_init(bars.q_full, 1);
@@ -148,6 +165,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bars.pv_done[t], 1);
         }
         mbar_init(bars.o_final, 1);
+        mbar_init(bars.count_ready, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -171,31 +189,44 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
+        bool ok = true;
+        auto load_kv = [&](int j) {   // K and V tile j into ring stage j % kStages (lane 0)
+            const int st = j % C::kStages;
+            const uint32_t use = j / C::kStages;
+            if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, abort_flag);
+            if (!ok) return;
+            mbar_arrive_expect_tx(&bars.k_full[st], C::kTileBytes);
+            for (int p = 0; p < C::kPanels; ++p)
+                tma_load_3d(smem + C::kKOff + st * C::kTileBytes + p * C::kPanelBytes, &tm_k,
+                            &bars.k_full[st], p * 64, j * kTileN, bh);
+            issued_k = j + 1;
+            if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, abort_flag);
+            if (!ok) return;
+            mbar_arrive_expect_tx(&bars.v_full[st], C::kTileBytes);
+            for (int p = 0; p < C::kPanels; ++p)
+                tma_load_3d(smem + C::kVOff + st * C::kTileBytes + p * C::kPanelBytes, &tm_v,
+                            &bars.v_full[st], p * 64, j * kTileN, bh);
+            issued_v = j + 1;
+        };
         if (lane_id() == 0) {
-            bool ok = true;
             mbar_arrive_expect_tx(bars.q_full, kQTiles * C::kTileBytes);
             for (int t = 0; t < kQTiles; ++t)
                 for (int p = 0; p < C::kPanels; ++p)
                     tma_load_3d(smem + C::kQOff + t * C::kTileBytes + p * C::kPanelBytes, &tm_q,
                                 bars.q_full, p * 64, row0 + t * kTileM, bh);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int st = j % C::kStages;
-                const uint32_t use = j / C::kStages;
-                if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bars.k_full[st], C::kTileBytes);
-                for (int p = 0; p < C::kPanels; ++p)
-                    tma_load_3d(smem + C::kKOff + st * C::kTileBytes + p * C::kPanelBytes, &tm_k,
-                                &bars.k_full[st], p * 64, j * kTileN, bh);
-                issued_k = j + 1;
-                if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bars.v_full[st], C::kTileBytes);
-                for (int p = 0; p < C::kPanels; ++p)
-                    tma_load_3d(smem + C::kVOff + st * C::kTileBytes + p * C::kPanelBytes, &tm_v,
-                                &bars.v_full[st], p * 64, j * kTileN, bh);
-                issued_v = j + 1;
+            load_kv(0);
+        }
+        __syncwarp();
+        int n_kv = n_kv_all;
+        if constexpr (kHasBias) {
+            n_kv = live_key_tiles(key_bias + static_cast<size_t>(bh / H) * S, S);
+            if (lane_id() == 0) {
+                *n_live_slot = n_kv;
+                mbar_arrive(bars.count_ready);   // release: the count is visible to the waiters
             }
+        }
+        if (lane_id() == 0) {
+            for (int j = 1; j < n_kv && ok; ++j) load_kv(j);
             // on an abort (here or in another role) the copies are drained at teardown
         }
         __syncwarp();
@@ -244,6 +275,11 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 issue_qk(1, 0);
                 tc_commit(&bars.s_full[1]);
                 tc_commit(&bars.k_empty[0]);
+            }
+            int n_kv = n_kv_all;
+            if constexpr (kHasBias) {
+                if (ok) ok = mbar_wait(bars.count_ready, 0, abort_flag);
+                n_kv = *n_live_slot;
             }
             if constexpr (C::kSepP) {
                 // Fixed issue order per key tile j, the order in which the softmax warpgroups
@@ -340,6 +376,11 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         float m_run = -INFINITY;   // running max, log2 units (scale folded in)
         float l_run = 0.f;         // running sum over this warp's half of the columns
         bool ok = true;
+        int n_kv = n_kv_all;
+        if constexpr (kHasBias) {
+            ok = mbar_wait_warp(bars.count_ready, 0, abort_flag);
+            n_kv = *n_live_slot;
+        }
         // publish v in slot `buf` and read the partner half's value once both are in
         auto exchange = [&](float v, int buf, uint32_t phase, float* other) -> bool {
             *xslot(buf, hf) = v;
@@ -353,7 +394,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             return true;
         };
 
-        for (int j = 0; j < n_kv; ++j) {
+        for (int j = 0; ok && j < n_kv; ++j) {
             ok = mbar_wait_warp(&bars.s_full[t], j & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();

@@ -203,3 +203,45 @@ def test_all_scores_far_below_zero(D, S):
     assert s_max < -1000.0, s_max                     # the case is what it claims
     assert_bf16_parity(got, ref, 2, "scores far below zero")
 
+
+
+def test_key_bias_trailing_masked_tiles_are_skipped_bit_exactly():
+    """Key tiles holding only -inf-biased keys (right padding) are never read: rows of a
+    640-key problem whose keys 384.. carry -inf equal, bit for bit, the same rows of the
+    384-key problem, even with NaN K and V in the skipped tiles."""
+    B_, H, S, Sl, D = 2, 3, 640, 384, 64
+    c = syn.encoder_case(B_, H, S, D, seed=97)
+    kb = torch.zeros((B_, S), dtype=torch.float32)
+    kb[:, Sl:] = float("-inf")
+    k = c.k.clone()
+    v = c.v.clone()
+    k[:, :, Sl:] = float("nan")
+    v[:, :, Sl:] = float("nan")
+    q_d, k_d, v_d = (t.to(DEV) for t in (c.q, k, v))
+    full = B.attn_encoder_fwd(q_d, k_d, v_d, c.softmax_scale, key_bias=kb.to(DEV))
+    q_t, k_t, v_t = (t[:, :, :Sl].contiguous().to(DEV) for t in (c.q, k, v))
+    kb_t = torch.zeros((B_, Sl), dtype=torch.float32, device=DEV)
+    short = B.attn_encoder_fwd(q_t, k_t, v_t, c.softmax_scale, key_bias=kb_t)
+    assert B.attn_check() == 0
+    assert torch.isfinite(full.float()).all()
+    assert torch.equal(full[:, :, :Sl], short)
+    ref = oracle.encoder_attention(to_f64(c.q), to_f64(k), to_f64(v), c.softmax_scale,
+                                   key_bias=kb.double().numpy())
+    assert_bf16_parity(full, ref, 2, "trailing masked tiles")
+
+
+@pytest.mark.parametrize("lengths", [[1, 640], [129, 300], [640, 640]])
+def test_key_bias_ragged_lengths_per_batch_entry(lengths):
+    """Per batch entry a different number of kept keys (1 key, one tile and a bit, all):
+    each entry skips its own trailing tiles."""
+    S = 640
+    c = syn.encoder_case(len(lengths), 2, S, 64, seed=98 + lengths[0])
+    kb = torch.zeros((len(lengths), S), dtype=torch.float32)
+    for i, L in enumerate(lengths):
+        kb[i, L:] = float("-inf")
+    q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
+    got = B.attn_encoder_fwd(q, k, v, c.softmax_scale, key_bias=kb.to(DEV))
+    assert B.attn_check() == 0
+    ref = oracle.encoder_attention(to_f64(c.q), to_f64(c.k), to_f64(c.v), c.softmax_scale,
+                                   key_bias=kb.double().numpy())
+    assert_bf16_parity(got, ref, 2, f"lengths {lengths}")
