@@ -4,7 +4,8 @@
 // q/k/v/out in [B, H, S, D] bf16, D in {64, 128}: the attention core of the
 // ViT / NewBERT encoder pages ("V-JEPA2 ViT-L Encoder NKI Kernels for AWS
 // Trainium2", "vit-encoder-neuron-kernels": bidirectional self-attention with
-// head_dim 64 or 128; "gte-encoder-neuron-kernels": right-padding mask).
+// head_dim 64 or 128; "gte-encoder-neuron-kernels": right-padding mask). The library runs it
+// for D = 128 and for any call with a key bias; D = 64 without one goes to encoder1q.cuh.
 //
 // How (B200 design, not the pages' SBUF/PSUM one):
 //   * one CTA owns 2 query tiles of 128 rows of one (b, h) and streams the
@@ -23,7 +24,9 @@
 //     max grew by more than 2^8 (the final O / l uses the same m, so a stale m
 //     is exact). At D = 64 one column pair in eight takes 2^x from an FMA-pipe
 //     polynomial instead of the MUFU unit;
-//   * warp 16 (one elected thread) is the TMA producer.
+//   * warp 16 (one elected thread) is the TMA producer; with a key bias the whole warp
+//     also counts the key tiles up to the batch entry's last kept key, and the tiles
+//     after it (right padding) are neither loaded nor computed.
 // The two query tiles ping-pong: while one warpgroup computes exponentials the
 // tensor core runs the other tile's MMAs.
 #pragma once
@@ -44,8 +47,8 @@ constexpr int kSoftmaxWarps = 16;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
-// Of every 8 column pairs of an unmasked S tile, this many take 2^x from the FMA-pipe
-// polynomial instead of the MUFU ex2 unit. At D = 64 the exponentials are as many per
+// Of every 8 column pairs of an S tile on the unbiased path, this many take 2^x from the
+// FMA-pipe polynomial instead of the MUFU ex2 unit. At D = 64 the exponentials are as many per
 // MMA flop as MUFU can barely sustain, so a share moves to the FMA pipe (measured on the
 // ViT-L case: 0/8 35.2 us, 1/8 30.3 us, 2/8 30.6 us per call); at D = 128 the same 1/8
 // share measured 1% faster than none.
