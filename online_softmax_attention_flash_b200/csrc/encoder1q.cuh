@@ -8,9 +8,10 @@
 //
 // How. A CTA owns 128 query rows of one (b, h) and streams the key sequence in 128-key
 // tiles through a 2-stage TMA ring: warp 5 (one thread) issues QK(j+1) as soon as the
-// softmax has read S(j) and PV(j) once P(j) is written; warps 0-3 are the softmax, one
-// thread per row holding all 128 scores of its row, so the row max needs no exchange
-// between warps. TMEM holds S (128 columns), O (64) and P (64, bf16 pairs): 256 columns,
+// softmax has read S(j), and PV(j) in four 32-key parts, each as soon as the softmax warps
+// have written that chunk of P(j) (one completion commit per tile: a commit per part costs
+// more than the finer waits it would allow); warps 0-3 are the softmax, one thread per row
+// holding all 128 scores of its row, so the row max needs no exchange between warps. TMEM holds S (128 columns), O (64) and P (64, bf16 pairs): 256 columns,
 // and the CTA needs ~81 KB of shared memory, so two CTAs share an SM. The two query tiles
 // an SM works on then belong to different CTAs: nothing in the issue order couples their
 // phases, and one CTA's exponentials (MUFU) overlap the other's max, stores and waits.
@@ -41,9 +42,10 @@ constexpr int kQOff = 0;
 constexpr int kKOff = kQOff + kTileBytes;
 constexpr int kVOff = kKOff + kStages * kTileBytes;
 constexpr int kBarOff = kVOff + kStages * kTileBytes;
-// q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full, s_free, p_ready, pv_done,
+// q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full, s_free, p_ready[4], pv_done,
 // o_final, mma_done
-constexpr int kNumBars = 1 + 4 * kStages + 6;
+constexpr int kPChunks = kTileN / 32;   // P is written, and P.V issued, in 32-key chunks
+constexpr int kNumBars = 1 + 4 * kStages + 5 + kPChunks;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kMiscOff + 16 + 1024;
 
@@ -61,7 +63,7 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* s_full = v_empty + kStages;
     uint64_t* s_free = s_full + 1;
     uint64_t* p_ready = s_free + 1;
-    uint64_t* pv_done = p_ready + 1;
+    uint64_t* pv_done = p_ready + kPChunks;
     uint64_t* o_final = pv_done + 1;
     uint64_t* mma_done = o_final + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
@@ -82,7 +84,7 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         mbar_init(s_full, 1);
         mbar_init(s_free, 4);    // one arrival per softmax warp
-        mbar_init(p_ready, 4);
+        for (int c = 0; c < kPChunks; ++c) mbar_init(&p_ready[c], 4);
         mbar_init(pv_done, 1);
         mbar_init(o_final, 1);
         mbar_init(mma_done, 1);
@@ -142,10 +144,10 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_f16_ss(tmem_base + kColS, dq + 2 * kk, ka + 2 * kk, idesc_qk, kk > 0);
             };
-            auto issue_pv = [&](int st, bool acc) {
+            auto issue_pv = [&](int st, int c, bool acc) {   // keys 32 c .. 32 c + 31
                 const uint64_t va = dv + static_cast<uint64_t>((st * kTileBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk)
+                for (int kk = 2 * c; kk < 2 * c + 2; ++kk)
                     mma_f16_ts(tmem_base + kColO, tmem_base + kColP + kk * 8,
                                va + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                                (acc || kk > 0) ? 1u : 0u);
@@ -169,11 +171,14 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tc_commit(&k_empty[stn]);
                 }
                 const int st = j % kStages;
-                ok = mbar_wait(p_ready, j & 1, abort_flag) &&
-                     mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag);
+                ok = mbar_wait(&v_full[st], (j / kStages) & 1, abort_flag);
+                for (int c = 0; c < kPChunks && ok; ++c) {   // each chunk as soon as it is in
+                    ok = mbar_wait(&p_ready[c], j & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(st, c, j > 0);
+                }
                 if (!ok) break;
-                tc_fence_after();
-                issue_pv(st, j > 0);
                 tc_commit(pv_done);
                 tc_commit(&v_empty[st]);
             }
@@ -233,7 +238,7 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const float alpha = upd ? ex2_approx(m_run - m_use) : 1.f;
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int c = 0; c < kTileN / 32; ++c) {
+            for (int c = 0; c < kPChunks; ++c) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
@@ -251,35 +256,42 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     else acc0 = __fadd2_rn(acc0, pv);
                     pk[k] = pack_bf16x2(pv.x, pv.y);
                 }
-                // P and O are free once PV of the previous tile has completed
                 if (c == 0 && j > 0) {
+                    // P and O are free once PV of the previous tile has completed; O is
+                    // rescaled now, before any part of PV(j) can be issued
                     if (!__all_sync(0xffffffffu, pv_seen)) {
                         ok = mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag);
                         if (!ok) break;
                     }
                     tc_fence_after();
+                    if (__any_sync(0xffffffffu, upd)) {
+#pragma unroll 1
+                        for (int h = 0; h < kD / 16; ++h) {
+                            uint32_t w[16];
+                            tmem_ld16_wait(tO + h * 16, w);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                            tmem_st16(tO + h * 16, w);
+                        }
+                    }
+                }
+                if (c > 0) {   // chunk c - 1 (and the O rescale) is in TMEM: PV may read it
+                    tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane_id() == 0) mbar_arrive(&p_ready[c - 1]);
                 }
                 // QK(j+1) was issued when S(j) had been read: look now whether S(j+1) is in
-                if (c == kTileN / 32 - 1) s_seen = j + 1 < n_kv && mbar_test(s_full, (j + 1) & 1);
+                if (c == kPChunks - 1) s_seen = j + 1 < n_kv && mbar_test(s_full, (j + 1) & 1);
                 tmem_st16(tP + c * 16, pk);
             }
             if (!ok) break;
             l_run = l_run * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
             m_run = m_next;
-            if (j > 0 && __any_sync(0xffffffffu, upd)) {
-#pragma unroll
-                for (int c = 0; c < kD / 32; ++c) {
-                    uint32_t w[32];
-                    tmem_ld32_wait(tO + c * 32, w);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-                    tmem_st32(tO + c * 32, w);
-                }
-            }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane_id() == 0) mbar_arrive(p_ready);
+            if (lane_id() == 0) mbar_arrive(&p_ready[kPChunks - 1]);
         }
         if (ok) ok = mbar_wait_warp(o_final, 0, abort_flag);
         if (ok) {
