@@ -16,13 +16,27 @@
 // an SM works on then belong to different CTAs: nothing in the issue order couples their
 // phases, and one CTA's exponentials (MUFU) overlap the other's max, stores and waits.
 // The running max may be stale by up to 2^8 (the final O / l uses the same reference);
-// two column pairs in eight take 2^x from the FMA-pipe polynomial.
+// two column pairs in eight take 2^x from the FMA-pipe polynomial. Each thread loads its
+// row of S in two 64-column halves: the max of the first half overlaps the load of the
+// second (four quarters were slower).
 #pragma once
 
 #include "ptx.cuh"
 
 namespace attn {
 namespace enc1q {
+
+// 64 columns of this warp's 32 TMEM lanes, left in flight (tc_wait_ld64 completes them)
+__device__ __forceinline__ void tmem_ld64_async(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+                 : "r"(taddr)
+                 : "memory");
+}
+// waits for the warp's TMEM loads; r is named so that no read of it moves above the wait
+__device__ __forceinline__ void tc_wait_ld64(uint32_t (&r)[64]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63]) :: "memory");
+}
 
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
@@ -205,27 +219,43 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int kv0 = j * kTileN;
             const int valid = S - kv0;
             uint32_t u[kTileN];
-            tmem_ld128_wait(tS, u);
+            uint32_t (&ua)[64] = *reinterpret_cast<uint32_t(*)[64]>(u);
+            uint32_t (&ub)[64] = *reinterpret_cast<uint32_t(*)[64]>(u + 64);
+            tmem_ld64_wait(tS, ua);
+            tmem_ld64_async(tS + 64, ub);   // the second half lands while the first is maxed
+            // raw scores (scale folded into the exponent); columns past S are -inf
+            if (valid < 64) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (i >= valid) u[i] = __float_as_uint(-INFINITY);
+            }
+            // pairs first, then three-input maxes over groups of 8 columns
+            static_assert(kTileN == 128, "the row is loaded and maxed in two halves of 64");
+            float mx[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                mx[e] = fmaxf(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+#pragma unroll
+            for (int i = 8; i < 64; i += 8) {
+                mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+                mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
+                mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
+                mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
+            }
+            tc_wait_ld64(ub);
             tc_fence_before();     // S may be overwritten by QK(j+1) from here on
             __syncwarp();
             if (lane_id() == 0) mbar_arrive(s_free);
             // PV(j-1) was issued when P(j-1) was complete and has most likely finished: look
             // now, use the answer before P(j) is stored
             const bool pv_seen = j == 0 || mbar_test(pv_done, (j - 1) & 1);
-            // raw scores (scale folded into the exponent); columns past S are -inf
             if (valid < kTileN) {
 #pragma unroll
-                for (int i = 0; i < kTileN; ++i)
+                for (int i = 64; i < kTileN; ++i)
                     if (i >= valid) u[i] = __float_as_uint(-INFINITY);
             }
-            // pairs first, then three-input maxes over groups of 8 columns
-            static_assert(kTileN % 8 == 0, "row max reads whole groups of 8 columns");
-            float mx[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                mx[e] = fmaxf(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-#pragma unroll
-            for (int i = 8; i < kTileN; i += 8) {
+            for (int i = 64; i < kTileN; i += 8) {
                 mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
                 mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
                 mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
