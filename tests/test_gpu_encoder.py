@@ -44,11 +44,30 @@ def test_vitl_b1_h16_s2048_d64(layer):
     assert_bf16_parity(_run(case), _oracle(case), 2, f"vitl layer {layer}")
 
 
-@pytest.mark.parametrize("S", [1, 7, 64, 127, 128, 129, 255, 256, 257, 300, 513])
+@pytest.mark.parametrize("S", [1, 7, 63, 64, 65, 127, 128, 129, 192, 193, 255, 256, 257, 300, 513])
 @pytest.mark.parametrize("D", [64, 128])
 def test_ragged_lengths(S, D):
     case = syn.encoder_case(2, 3, S, D, seed=300 + S + D, softmax_scale=D ** -0.5)
     assert_bf16_parity(_run(case), _oracle(case), 2, f"S={S} D={D}")
+
+
+@pytest.mark.parametrize("D,with_bias", [(64, False), (64, True), (128, False)])
+def test_running_max_grows_across_key_tiles(D, with_bias):
+    """Scores that climb from one 128-key tile to the next (the keys of tile t carry 8 t times
+    a direction the queries share), so the running max moves by more than 2^8 several times
+    after the first tile and O is rescaled in later tiles. A skipped rescale or a wrong factor
+    would leave the earlier tiles' share of O off by 2^8 or more."""
+    g = torch.Generator().manual_seed(4242 + D)
+    nb, nh, S = 2, 2, 700
+    w = torch.randn(D, generator=g)
+    w = w / w.norm()
+    tile = (torch.arange(S) // 128).float()
+    q = (torch.randn(nb, nh, S, D, generator=g) * 0.3 + 3.0 * w).to(torch.bfloat16)
+    k = (torch.randn(nb, nh, S, D, generator=g) * 0.3 + (8.0 * tile)[:, None] * w).to(torch.bfloat16)
+    v = torch.randn(nb, nh, S, D, generator=g).to(torch.bfloat16)
+    kb = (torch.rand((nb, S), generator=g) * 0.5).float() if with_bias else None
+    case = syn.EncoderCase(q, k, v, 0.125, kb)
+    assert_bf16_parity(_run(case), _oracle(case), 2, f"growing max D={D} bias={with_bias}")
 
 
 def test_head_dim_128_long():
