@@ -246,9 +246,8 @@ class EncoderWork:
         self.launches_per_step = cfg["sets"]
         self.work_per_step = self.flops_per_launch * cfg["sets"]
         self.unit, self.bound = "TFLOP/s", "tensor"
-        # head dim 64 without a key bias runs the one-query-tile kernel
-        self.kernel_regex = ("encoder_1q_kernel" if D == 64 and self.bias[0] is None
-                             else "encoder_fwd_kernel")
+        # head dim 64 (with or without a key bias) runs the one-query-tile kernel
+        self.kernel_regex = "encoder_1q_kernel" if D == 64 else "encoder_fwd_kernel"
         self.peak_ratio = 1.0
         self.dtype = "bf16"
 

@@ -46,12 +46,14 @@ int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
     return ATTN_OK;
 }
 
-// Head dim 64 without a key bias: one query tile per CTA, two CTAs per SM (encoder1q.cuh).
+// Head dim 64: one query tile per CTA, two CTAs per SM (encoder1q.cuh), with or without a
+// key bias.
+template <bool kBias>
 int launch_encoder1q(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
-                     int H, int S, float scale, cudaStream_t stream) {
+                     int H, int S, float scale, const float* key_bias, cudaStream_t stream) {
     using namespace attn::enc1q;
     static std::atomic<uint64_t> smem_done{0};
-    auto kernel = encoder_1q_kernel;
+    auto kernel = encoder_1q_kernel<kBias>;
     int rc = ensure_smem(kernel, kSmemBytes, smem_done);
     if (rc) return rc;
     CUtensorMap tq, tk, tv;
@@ -61,8 +63,8 @@ int launch_encoder1q(const uint16_t* q, const uint16_t* k, const uint16_t* v, ui
     if ((rc = attn::encode_map_3d_bf16(&tk, k, kD, rows, heads, 64, kTileN))) return rc;
     if ((rc = attn::encode_map_3d_bf16(&tv, v, kD, rows, heads, 64, kTileN))) return rc;
     dim3 grid((S + kTileM - 1) / kTileM, static_cast<unsigned>(heads));
-    return attn::launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, out, S,
-                            scale * kLog2e);
+    return attn::launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, out,
+                            key_bias, H, S, scale * kLog2e);
 }
 
 template <int D, bool kBias>
@@ -180,8 +182,8 @@ int attn_encoder_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, ui
     if (key_bias && (reinterpret_cast<uintptr_t>(key_bias) & 3u)) return ATTN_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (D == 64)
-        return key_bias ? launch_encoder<64, true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
-                        : launch_encoder1q(q, k, v, out, B, H, S, softmax_scale, st);
+        return key_bias ? launch_encoder1q<true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
+                        : launch_encoder1q<false>(q, k, v, out, B, H, S, softmax_scale, nullptr, st);
     return key_bias ? launch_encoder<128, true>(q, k, v, out, B, H, S, softmax_scale, key_bias, st)
                     : launch_encoder<128, false>(q, k, v, out, B, H, S, softmax_scale, nullptr, st);
 }

@@ -1,29 +1,26 @@
-// encoder.cuh -- non-causal multi-head encoder attention forward for sm_100a.
+// encoder.cuh -- non-causal multi-head encoder attention forward at head_dim 128 (sm_100a).
 //
 // What it computes: out[b,h] = softmax(scale * Q K^T + key_bias[b]) V for
-// q/k/v/out in [B, H, S, D] bf16, D in {64, 128}: the attention core of the
-// ViT / NewBERT encoder pages ("V-JEPA2 ViT-L Encoder NKI Kernels for AWS
-// Trainium2", "vit-encoder-neuron-kernels": bidirectional self-attention with
-// head_dim 64 or 128; "gte-encoder-neuron-kernels": right-padding mask). The library runs it
-// for D = 128 and for any call with a key bias; D = 64 without one goes to encoder1q.cuh.
+// q/k/v/out in [B, H, S, 128] bf16: the attention core of the ViT / NewBERT encoder pages
+// ("V-JEPA2 ViT-L Encoder NKI Kernels for AWS Trainium2", "vit-encoder-neuron-kernels":
+// bidirectional self-attention with head_dim 64 or 128; "gte-encoder-neuron-kernels":
+// right-padding mask). Head dim 64 runs the one-query-tile kernel (encoder1q.cuh).
 //
 // How (B200 design, not the pages' SBUF/PSUM one):
 //   * one CTA owns 2 query tiles of 128 rows of one (b, h) and streams the
 //     whole key sequence in 128-key tiles through a TMA ring in shared memory;
 //   * warp 17 (one elected thread) issues tcgen05.mma: S_t = Q_t K^T into a
 //     TMEM fp32 accumulator per query tile, then O_t += P_t V with P_t read
-//     back from TMEM (bf16; in its own columns at D = 64, over S_t at D = 128)
-//     and O_t an fp32 TMEM accumulator. At D = 64 it issues in a fixed order per
-//     key tile j -- QK_0(j+1), PV_1(j-1), QK_1(j+1), PV_0(j) -- the order in
-//     which the two softmax warpgroups free their inputs;
+//     back from TMEM (bf16, written over S_t: S and O of both tiles fill TMEM)
+//     and O_t an fp32 TMEM accumulator;
 //   * warps 0-7 / 8-15 are the softmax warpgroups of query tiles 0 / 1: a row
 //     (one TMEM lane) is shared by two warps on the same scheduler, 64 S
 //     columns each, which exchange their halves' maxima and sums through
 //     shared memory; each keeps the running max m and sum l in fp32 registers,
 //     writes P, and rescales its half of the O row in TMEM only when the row
 //     max grew by more than 2^8 (the final O / l uses the same m, so a stale m
-//     is exact). At D = 64 one column pair in eight takes 2^x from an FMA-pipe
-//     polynomial instead of the MUFU unit;
+//     is exact); one column pair in eight takes 2^x from an FMA-pipe polynomial
+//     instead of the MUFU unit;
 //   * warp 16 (one elected thread) is the TMA producer; with a key bias the whole warp
 //     also counts the key tiles up to the batch entry's last kept key, and the tiles
 //     after it (right padding) are neither loaded nor computed.
@@ -48,42 +45,34 @@ constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
 // Of every 8 column pairs of an S tile on the unbiased path, this many take 2^x from the
-// FMA-pipe polynomial instead of the MUFU ex2 unit. At D = 64 the exponentials are as many per
-// MMA flop as MUFU can barely sustain, so a share moves to the FMA pipe (measured on the
-// ViT-L case: 0/8 35.2 us, 1/8 30.3 us, 2/8 30.6 us per call); at D = 128 the same 1/8
-// share measured 1% faster than none.
-template <int D>
-__host__ __device__ constexpr int poly_eighths() { return 1; }
+// FMA-pipe polynomial instead of the MUFU ex2 unit (one in eight measured 1% faster than none).
+constexpr int kPolyEighths = 1;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
+    static_assert(D == 128, "head dim 64 runs the one-query-tile kernel");
     static constexpr int kPanels = D / 64;              // 128-byte swizzle panels per row
     static constexpr int kPanelBytes = 128 * 128;       // 128 rows x 128 bytes
     static constexpr int kTileBytes = kPanels * kPanelBytes;
-    static constexpr int kStages = (D == 64) ? 4 : 2;
+    static constexpr int kStages = 2;
     static constexpr int kQOff = 0;
     static constexpr int kKOff = kQOff + kQTiles * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
     // o_final, xchg[2] (row-max / row-sum exchange between the two halves of a tile),
-    // s_free[2] (softmax has read S_t), pv_done[2] (PV_t has completed), count_ready (the
-    // number of key tiles with a kept key is known; key-bias kernels)
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 2 + 2 + 1;
+    // count_ready (the number of key tiles with a kept key is known; key-bias kernels)
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 1;
     static constexpr int kXchgOff = kBarOff + kNumBars * 8;   // float [2 buf][2 tile][2 half][128]
     static constexpr int kMiscOff = kXchgOff + 2 * 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + tmem slot, abort flag, alignment slack
-    // TMEM columns: S_t at 128 t, O_t at 256 + D t. For D = 64 the P tiles (bf16 pairs,
-    // 64 columns each) get their own columns at 384 + 64 t, so the next QK can overwrite
-    // S_t as soon as the softmax has read it; for D = 128 TMEM is full and P_t is written
-    // over the first 64 columns of S_t.
+    // TMEM columns: S_t at 128 t, O_t at 256 + D t. TMEM is full, so P_t (bf16 pairs) is
+    // written over the first 64 columns of S_t.
     static constexpr uint32_t kColS0 = 0;
     static constexpr uint32_t kColO0 = 256;
-    static constexpr bool kSepP = (D == 64);
-    static constexpr uint32_t kColP0 = kSepP ? 256 + 2 * D : 0;
 };
 
 struct Bars {
@@ -96,8 +85,6 @@ struct Bars {
     uint64_t* p_ready;
     uint64_t* o_final;
     uint64_t* xchg;
-    uint64_t* s_free;
-    uint64_t* pv_done;
     uint64_t* count_ready;
 };
 
@@ -115,9 +102,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
     r.p_ready = r.s_full + 2;
     r.o_final = r.p_ready + 2;
     r.xchg = r.o_final + 1;
-    r.s_free = r.xchg + 2;
-    r.pv_done = r.s_free + 2;
-    r.count_ready = r.pv_done + 2;
+    r.count_ready = r.xchg + 2;
     return r;
 }
 
@@ -164,8 +149,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bars.s_full[t], 1);
             mbar_init(&bars.p_ready[t], kSoftmaxWarps / 2);   // one arrival per softmax warp of the tile
             mbar_init(&bars.xchg[t], kSoftmaxWarps / 2);
-            mbar_init(&bars.s_free[t], kSoftmaxWarps / 2);
-            mbar_init(&bars.pv_done[t], 1);
         }
         mbar_init(bars.o_final, 1);
         mbar_init(bars.count_ready, 1);
@@ -263,7 +246,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             auto issue_pv = [&](int t, int st, bool acc) {
                 const uint64_t va = dv + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
                 const uint32_t d = tmem_base + C::kColO0 + t * D;
-                const uint32_t a = C::kSepP ? tmem_base + C::kColP0 + t * 64 : tmem_base + C::kColS0 + t * 128;
+                const uint32_t a = tmem_base + C::kColS0 + t * 128;   // P_t over S_t
 #pragma unroll
                 for (int kk = 0; kk < kTileN / 16; ++kk)
                     mma_f16_ts(d, a + kk * 8, va + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
@@ -284,48 +267,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (ok) ok = mbar_wait(bars.count_ready, 0, abort_flag);
                 n_kv = *n_live_slot;
             }
-            if constexpr (C::kSepP) {
-                // Fixed issue order per key tile j, the order in which the softmax warpgroups
-                // free their inputs (tile 1 runs half a key tile behind tile 0):
-                //   QK_0(j+1) once tile 0 has read S_0(j); PV_1(j-1) once P_1(j-1) is written;
-                //   QK_1(j+1) once tile 1 has read S_1(j); PV_0(j) once P_0(j) is written.
-                // Every wait is on a barrier whose producer depends only on MMAs issued
-                // earlier in this order. A K stage is released after QK_1 has used it, a V
-                // stage after PV_1.
-                auto pv = [&](int t, int j) -> bool {
-                    const int sp = j % C::kStages;
-                    if (!mbar_wait(&bars.p_ready[t], j & 1, abort_flag)) return false;
-                    if (!mbar_wait(&bars.v_full[sp], (j / C::kStages) & 1, abort_flag)) return false;
-                    tc_fence_after();
-                    issue_pv(t, sp, j > 0);
-                    tc_commit(&bars.pv_done[t]);
-                    if (t == 1) tc_commit(&bars.v_empty[sp]);
-                    return true;
-                };
-                for (int j = 0; j < n_kv && ok; ++j) {
-                    const bool more = j + 1 < n_kv;
-                    const int stn = (j + 1) % C::kStages;
-                    if (more) {
-                        ok = mbar_wait(&bars.s_free[0], j & 1, abort_flag) &&
-                             mbar_wait(&bars.k_full[stn], ((j + 1) / C::kStages) & 1, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_qk(0, stn);
-                        tc_commit(&bars.s_full[0]);
-                    }
-                    if (j > 0 && !(ok = pv(1, j - 1))) break;
-                    if (more) {
-                        ok = mbar_wait(&bars.s_free[1], j & 1, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_qk(1, stn);
-                        tc_commit(&bars.s_full[1]);
-                        tc_commit(&bars.k_empty[stn]);
-                    }
-                    ok = pv(0, j);
-                }
-                if (ok) ok = pv(1, n_kv - 1);
-            } else {
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j % C::kStages;
                 const uint32_t ph = (j / C::kStages) & 1;
@@ -355,7 +296,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 tc_commit(&bars.v_empty[st]);
             }
-            }
             // o_final fires when every MMA above has completed (committed on the abort path
             // too: teardown waits for it before TMEM is freed)
             tc_commit(bars.o_final);
@@ -370,7 +310,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem_base + lane_off + C::kColS0 + t * 128;
         const uint32_t tSh = tS + hf * kHalf;            // this warp's S columns
-        const uint32_t tPh = (C::kSepP ? tmem_base + lane_off + C::kColP0 + t * 64 : tS) + hf * (kHalf / 2);
+        const uint32_t tPh = tS + hf * (kHalf / 2);    // this warp's P columns (over S)
         const uint32_t tOh = tmem_base + lane_off + C::kColO0 + t * D + hf * (D / 2);
         float* xchg = reinterpret_cast<float*>(smem + C::kXchgOff);
         auto xslot = [&](int buf, int half) { return xchg + ((buf * 2 + t) * 2 + half) * kTileM + r; };
@@ -426,11 +366,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                 for (int i = 0; i < kHalf; ++i)
                     if (col0 + i >= valid) u[i] = __float_as_uint(-INFINITY);
-            }
-            if constexpr (C::kSepP) {   // S_t may be overwritten by the next QK from here on
-                tc_fence_before();
-                __syncwarp();
-                if (lane_id() == 0) mbar_arrive(&bars.s_free[t]);
             }
             float m_half;
             if (raw_path) {
@@ -500,7 +435,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                                     make_float2(-m_use, -m_use));
                         // the polynomial also takes the -inf columns past S of a ragged tile:
                         // it clamps them to 2^-125, and their V rows are zero-filled
-                        if ((kk & 7) < poly_eighths<D>()) pv = exp2_poly2(x);
+                        if ((kk & 7) < kPolyEighths) pv = exp2_poly2(x);
                         else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     } else {
                         pv = make_float2(ex2_approx(sv.x - m_use), ex2_approx(sv.y - m_use));
@@ -509,15 +444,7 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     else acc0 = __fadd2_rn(acc0, pv);
                     pk[k] = pack_bf16x2(pv.x, pv.y);
                 }
-                // With separate P columns, P_t and O_t are free only once PV_t of the
-                // previous tile has completed (with P over S, s_full already implied it).
-                if constexpr (C::kSepP) {
-                    if (c == 0 && j > 0) {
-                        ok = mbar_wait_warp(&bars.pv_done[t], (j - 1) & 1, abort_flag);
-                        if (!ok) break;   // PV_t(j-1) may still read P_t: leave it alone
-                        tc_fence_after();
-                    }
-                }
+                // P over S: s_full of this tile implied that PV_t of the previous one is done.
                 // Both halves read their S columns before the exchange above, so P columns
                 // that overlap the first half's S columns are free to write.
                 tmem_st16(tPh + c * 16, pk);

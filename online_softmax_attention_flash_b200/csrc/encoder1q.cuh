@@ -1,10 +1,14 @@
 // encoder1q.cuh -- non-causal encoder attention forward at head_dim 64, one query tile per
 // CTA, two CTAs per SM (sm_100a).
 //
-// What it computes: the same as encoder_fwd_kernel (encoder.cuh) for D = 64 without a key
-// bias: out[b,h] = softmax(scale * Q K^T) V, q/k/v/out [B, H, S, 64] bf16. (With a key bias
-// the two-tile kernel runs: a bias on 128 columns per thread costs registers this kernel,
-// at two CTAs per SM, does not have.)
+// What it computes: the same as encoder_fwd_kernel (encoder.cuh), at D = 64: out[b,h] =
+// softmax(scale * Q K^T + key_bias[b]) V, q/k/v/out [B, H, S, 64] bf16, key_bias [B, S] fp32
+// additive or none. With a key bias (kHasBias) the producer counts the key tiles up to the
+// entry's last kept key while the first copies fly (the tiles after it are never loaded);
+// a tile whose bias is zero over its columns takes the unbiased path, any other tile turns
+// its scores into biased log2-unit scores before the max, and a dropped key (bias -inf)
+// weighs exactly 0 wherever the polynomial would give 2^-125, since its V row may hold any
+// finite value.
 //
 // How. A CTA owns 128 query rows of one (b, h) and streams the key sequence in 128-key
 // tiles through a 2-stage TMA ring: warp 5 (one thread) issues QK(j+1) as soon as the
@@ -57,16 +61,28 @@ constexpr int kKOff = kQOff + kTileBytes;
 constexpr int kVOff = kKOff + kStages * kTileBytes;
 constexpr int kBarOff = kVOff + kStages * kTileBytes;
 // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full, s_free, p_ready[4], pv_done,
-// o_final, mma_done
+// o_final, mma_done, count_ready
 constexpr int kPChunks = kTileN / 32;   // P is written, and P.V issued, in 32-key chunks
-constexpr int kNumBars = 1 + 4 * kStages + 5 + kPChunks;
-constexpr int kMiscOff = kBarOff + kNumBars * 8;
+constexpr int kNumBars = 1 + 4 * kStages + 6 + kPChunks;
+constexpr int kMiscOff = kBarOff + kNumBars * 8;   // TMEM address, abort flag, live tile count
 constexpr int kSmemBytes = kMiscOff + 16 + 1024;
 
+// Key tiles up to the last key whose bias is not -inf (at least one), found by a whole warp:
+// with right padding the trailing tiles hold only -inf keys, which take no part in any row.
+__device__ __forceinline__ int live_key_tiles(const float* kb, int S) {
+    int last = -1;
+    for (int c = static_cast<int>(lane_id()); c < S; c += 32)
+        if (__ldg(kb + c) != -INFINITY) last = c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    return max(1, (last + kTileN) / kTileN);
+}
+
+template <bool kHasBias>
 __global__ void __launch_bounds__(kThreads, 2)
 encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int S,
-                  float scale_log2) {
+                  const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out,
+                  const float* __restrict__ key_bias, int H, int S, float scale_log2) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + kBarOff);
@@ -80,13 +96,17 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* pv_done = p_ready + kPChunks;
     uint64_t* o_final = pv_done + 1;
     uint64_t* mma_done = o_final + 1;
+    uint64_t* count_ready = mma_done + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 4);
+    // with a key bias: the key tiles that hold a kept key (the producer counts them while the
+    // first copies fly and publishes the count through count_ready)
+    volatile int* n_live_slot = reinterpret_cast<volatile int*>(smem + kMiscOff + 8);
 
     const int warp = threadIdx.x >> 5;
     const int bh = blockIdx.y;
     const int row0 = blockIdx.x * kTileM;
-    const int n_kv = (S + kTileN - 1) / kTileN;
+    const int n_kv_all = (S + kTileN - 1) / kTileN;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -102,6 +122,7 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(pv_done, 1);
         mbar_init(o_final, 1);
         mbar_init(mma_done, 1);
+        mbar_init(count_ready, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -124,25 +145,37 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
+        bool ok = true;
+        auto load_kv = [&](int j) {   // K and V tile j into ring stage j % kStages (lane 0)
+            const int st = j % kStages;
+            const uint32_t use = j / kStages;
+            if (use > 0) ok = mbar_wait(&k_empty[st], (use - 1) & 1, abort_flag);
+            if (!ok) return;
+            mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+            tma_load_3d(smem + kKOff + st * kTileBytes, &tm_k, &k_full[st], 0, j * kTileN, bh);
+            issued_k = j + 1;
+            if (use > 0) ok = mbar_wait(&v_empty[st], (use - 1) & 1, abort_flag);
+            if (!ok) return;
+            mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+            tma_load_3d(smem + kVOff + st * kTileBytes, &tm_v, &v_full[st], 0, j * kTileN, bh);
+            issued_v = j + 1;
+        };
         if (lane_id() == 0) {
-            bool ok = true;
             mbar_arrive_expect_tx(q_full, kTileBytes);
             tma_load_3d(smem + kQOff, &tm_q, q_full, 0, row0, bh);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int st = j % kStages;
-                const uint32_t use = j / kStages;
-                if (use > 0) ok = mbar_wait(&k_empty[st], (use - 1) & 1, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&k_full[st], kTileBytes);
-                tma_load_3d(smem + kKOff + st * kTileBytes, &tm_k, &k_full[st], 0, j * kTileN, bh);
-                issued_k = j + 1;
-                if (use > 0) ok = mbar_wait(&v_empty[st], (use - 1) & 1, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-                tma_load_3d(smem + kVOff + st * kTileBytes, &tm_v, &v_full[st], 0, j * kTileN, bh);
-                issued_v = j + 1;
+            load_kv(0);
+        }
+        __syncwarp();
+        int n_kv = n_kv_all;
+        if constexpr (kHasBias) {
+            n_kv = live_key_tiles(key_bias + static_cast<size_t>(bh / H) * S, S);
+            if (lane_id() == 0) {
+                *n_live_slot = n_kv;
+                mbar_arrive(count_ready);   // release: the count is visible to the waiters
             }
         }
+        if (lane_id() == 0)
+            for (int j = 1; j < n_kv && ok; ++j) load_kv(j);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -172,6 +205,11 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 issue_qk(0);
                 tc_commit(s_full);
                 tc_commit(&k_empty[0]);
+            }
+            int n_kv = n_kv_all;
+            if constexpr (kHasBias) {
+                if (ok) ok = mbar_wait(count_ready, 0, abort_flag);
+                n_kv = *n_live_slot;
             }
             for (int j = 0; j < n_kv && ok; ++j) {
                 if (j + 1 < n_kv) {   // S(j+1) once the softmax has read S(j)
@@ -209,8 +247,13 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t tP = tmem_base + lane_off + kColP;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
+        int n_kv = n_kv_all;
+        if constexpr (kHasBias) {
+            ok = mbar_wait_warp(count_ready, 0, abort_flag);
+            n_kv = *n_live_slot;
+        }
         bool s_seen = false;   // S(j) already reported complete by an earlier look
-        for (int j = 0; j < n_kv; ++j) {
+        for (int j = 0; ok && j < n_kv; ++j) {
             if (!__all_sync(0xffffffffu, s_seen)) {
                 ok = mbar_wait_warp(s_full, j & 1, abort_flag);
                 if (!ok) break;
@@ -218,50 +261,105 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_after();
             const int kv0 = j * kTileN;
             const int valid = S - kv0;
+            bool raw_path = true;   // scores taken as they are (no key bias on this tile)
+            const float* kb = nullptr;
+            if constexpr (kHasBias) {
+                // A tile whose bias is zero over its columns before S is computed exactly as
+                // without a bias (with right padding: every tile but the one that holds the
+                // end of the entry's keys).
+                // (these loads also bring the tile's bias row into L1 ahead of the biased path;
+                // a per-tile bit from the producer's scan instead was 8% slower on a finite
+                // bias and gained only on an all-zero one)
+                kb = key_bias + static_cast<size_t>(bh / H) * S + kv0;
+                const int c = 4 * static_cast<int>(lane_id());
+                bool zero = true;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) zero = zero && (c + e >= valid || __ldg(kb + c + e) == 0.f);
+                raw_path = __all_sync(0xffffffffu, zero);
+            }
             uint32_t u[kTileN];
             uint32_t (&ua)[64] = *reinterpret_cast<uint32_t(*)[64]>(u);
             uint32_t (&ub)[64] = *reinterpret_cast<uint32_t(*)[64]>(u + 64);
-            tmem_ld64_wait(tS, ua);
-            tmem_ld64_async(tS + 64, ub);   // the second half lands while the first is maxed
-            // raw scores (scale folded into the exponent); columns past S are -inf
-            if (valid < 64) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (i >= valid) u[i] = __float_as_uint(-INFINITY);
-            }
-            // pairs first, then three-input maxes over groups of 8 columns
             static_assert(kTileN == 128, "the row is loaded and maxed in two halves of 64");
             float mx[4];
+            float m_tile;
+            bool pv_seen = true;
+            if (raw_path) {
+                tmem_ld64_wait(tS, ua);
+                tmem_ld64_async(tS + 64, ub);   // the second half lands while the first is maxed
+                // raw scores (scale folded into the exponent); columns past S are -inf
+                if (valid < 64) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                mx[e] = fmaxf(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+                    for (int i = 0; i < 64; ++i)
+                        if (i >= valid) u[i] = __float_as_uint(-INFINITY);
+                }
+                // pairs first, then three-input maxes over groups of 8 columns
 #pragma unroll
-            for (int i = 8; i < 64; i += 8) {
-                mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
-                mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
-                mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
-                mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
+                for (int e = 0; e < 4; ++e)
+                    mx[e] = fmaxf(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+#pragma unroll
+                for (int i = 8; i < 64; i += 8) {
+                    mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+                    mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
+                    mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
+                    mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
+                }
+                tc_wait_ld64(ub);
+                tc_fence_before();     // S may be overwritten by QK(j+1) from here on
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(s_free);
+                // PV(j-1) was issued when P(j-1) was complete and has most likely finished:
+                // look now, use the answer before P(j) is stored
+                pv_seen = j == 0 || mbar_test(pv_done, (j - 1) & 1);
+                if (valid < kTileN) {
+#pragma unroll
+                    for (int i = 64; i < kTileN; ++i)
+                        if (i >= valid) u[i] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int i = 64; i < kTileN; i += 8) {
+                    mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+                    mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
+                    mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
+                    mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
+                }
+                m_tile = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
+            } else if constexpr (kHasBias) {
+                tmem_ld64_wait(tS, ua);
+                tmem_ld64_wait(tS + 64, ub);
+                tc_fence_before();     // S may be overwritten by QK(j+1) from here on
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(s_free);
+                pv_seen = j == 0 || mbar_test(pv_done, (j - 1) & 1);
+                // biased score of column i in log2 units (scale folded in); -inf where the
+                // bias is -inf or past S; a finite bias stays finite (a -FLT_MAX fill keeps its
+                // key). Every lane reads the same biases: 16-byte broadcast loads.
+                mx[0] = mx[1] = mx[2] = mx[3] = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < kTileN; i += 4) {
+                    float4 b4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                    if (i + 3 < valid && ((reinterpret_cast<uintptr_t>(kb + i) & 15u) == 0)) {
+                        b4 = __ldg(reinterpret_cast<const float4*>(kb + i));
+                    } else {
+                        if (i < valid) b4.x = __ldg(kb + i);
+                        if (i + 1 < valid) b4.y = __ldg(kb + i + 1);
+                        if (i + 2 < valid) b4.z = __ldg(kb + i + 2);
+                        if (i + 3 < valid) b4.w = __ldg(kb + i + 3);
+                    }
+                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x = bb[e] == -INFINITY
+                                            ? -INFINITY
+                                            : fmaf(__uint_as_float(u[i + e]), scale_log2, fmaxf(bb[e] * kLog2e, -FLT_MAX));
+                        u[i + e] = __float_as_uint(x);
+                        mx[e] = fmaxf(mx[e], x);
+                    }
+                }
+                m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             }
-            tc_wait_ld64(ub);
-            tc_fence_before();     // S may be overwritten by QK(j+1) from here on
-            __syncwarp();
-            if (lane_id() == 0) mbar_arrive(s_free);
-            // PV(j-1) was issued when P(j-1) was complete and has most likely finished: look
-            // now, use the answer before P(j) is stored
-            const bool pv_seen = j == 0 || mbar_test(pv_done, (j - 1) & 1);
-            if (valid < kTileN) {
-#pragma unroll
-                for (int i = 64; i < kTileN; ++i)
-                    if (i >= valid) u[i] = __float_as_uint(-INFINITY);
-            }
-#pragma unroll
-            for (int i = 64; i < kTileN; i += 8) {
-                mx[0] = fmax3(mx[0], __uint_as_float(u[i]), __uint_as_float(u[i + 1]));
-                mx[1] = fmax3(mx[1], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
-                mx[2] = fmax3(mx[2], __uint_as_float(u[i + 4]), __uint_as_float(u[i + 5]));
-                mx[3] = fmax3(mx[3], __uint_as_float(u[i + 6]), __uint_as_float(u[i + 7]));
-            }
-            const float m_tile = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
+            // log2-unit factor of the scores in u: the scale on the raw path, 1 on the biased one
+            const float sc = raw_path ? scale_log2 : 1.f;
             const bool upd = m_tile > m_run + kRescaleThreshold;
             const float m_next = upd ? m_tile : m_run;
             const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
@@ -274,14 +372,20 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int k = 0; k < 16; ++k) {
                     const int kk = c * 16 + k;   // column pair index
                     const float2 sv = make_float2(__uint_as_float(u[2 * kk]), __uint_as_float(u[2 * kk + 1]));
-                    const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
-                                                make_float2(-m_use, -m_use));
+                    const float2 x = __ffma2_rn(sv, make_float2(sc, sc), make_float2(-m_use, -m_use));
                     float2 pv;
                     // the polynomial also takes the -inf columns of a ragged tile: it clamps
                     // them to 2^-125, and as past S the V rows are zero-filled they add
                     // nothing to O (and less than an ulp to the row sum)
-                    if ((kk & 7) < kPolyEighths) pv = exp2_poly2(x);
-                    else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    if ((kk & 7) < kPolyEighths) {
+                        pv = exp2_poly2(x);
+                        if constexpr (kHasBias) {   // a dropped key weighs exactly 0 (its V may hold anything finite)
+                            if (x.x == -INFINITY) pv.x = 0.f;
+                            if (x.y == -INFINITY) pv.y = 0.f;
+                        }
+                    } else {
+                        pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    }
                     if (k & 1) acc1 = __fadd2_rn(acc1, pv);
                     else acc0 = __fadd2_rn(acc0, pv);
                     pk[k] = pack_bf16x2(pv.x, pv.y);

@@ -58,8 +58,8 @@ def _until_timeout(lib, launch, tries=5):
     return seen
 
 
-@pytest.mark.parametrize("D,with_bias", [(64, False), (64, True), (128, False)],
-                         ids=["d64_one_tile", "d64_key_bias_two_tile", "d128_two_tile"])
+@pytest.mark.parametrize("D,with_bias", [(64, False), (64, True), (128, False), (128, True)],
+                         ids=["d64", "d64_key_bias", "d128", "d128_key_bias"])
 def test_encoder_wait_timeout_is_reported(short_wait_lib, D, with_bias):
     c = syn.encoder_case(1, 4, 1024, D, seed=501)
     q, k, v = (t.to(DEV) for t in (c.q, c.k, c.v))
