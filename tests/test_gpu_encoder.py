@@ -189,6 +189,25 @@ def test_general_finite_key_bias():
     assert_bf16_parity(out, ref, 2, "general key bias")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_dropped_keys_weigh_exactly_zero(D):
+    """Keys dropped by a -inf bias inside tiles that keep other keys: their V rows hold the
+    largest finite bf16 value, so any weight above 0 (2^-125 from the polynomial would already
+    give ~7) shows in the output; the result must match the oracle, which drops them."""
+    c = syn.encoder_case(2, 3, 600, D, seed=91, softmax_scale=D ** -0.5)
+    kb = torch.zeros((2, 600), dtype=torch.float32)
+    kb[:, 1::3] = float("-inf")          # every third key of every tile
+    kb[1, 450:] = float("-inf")          # and a padded tail in entry 1
+    v = c.v.clone()
+    big = torch.finfo(torch.bfloat16).max
+    v[:, :, 1::3, :] = big
+    v[1, :, 450:, :] = big
+    case = syn.EncoderCase(c.q, c.k, v, c.softmax_scale, kb)
+    out = _run(case)
+    assert torch.isfinite(out.float()).all()
+    assert_bf16_parity(out, _oracle(case), 2, f"dropped keys D={D}")
+
+
 def test_float32_min_key_bias_keeps_keys():
     # a finite -FLT_MAX bias keeps its keys: all of them give the mean of V, next to 0-biased
     # keys they carry no weight (-inf alone removes a key)
