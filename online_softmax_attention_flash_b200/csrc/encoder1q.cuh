@@ -260,22 +260,31 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             tc_fence_after();
             const int kv0 = j * kTileN;
-            const int valid = S - kv0;
+            int valid = S - kv0;    // columns of this tile that take part (the rest are -inf)
             bool raw_path = true;   // scores taken as they are (no key bias on this tile)
             const float* kb = nullptr;
             if constexpr (kHasBias) {
-                // A tile whose bias is zero over its columns before S is computed exactly as
-                // without a bias (with right padding: every tile but the one that holds the
-                // end of the entry's keys).
-                // (these loads also bring the tile's bias row into L1 ahead of the biased path;
-                // a per-tile bit from the producer's scan instead was 8% slower on a finite
-                // bias and gained only on an all-zero one)
+                // A tile whose bias is 0 on a prefix of its columns and -inf on the rest (no
+                // bias at all, or the end of a right-padded entry) is computed as without a
+                // bias, with the -inf part masked like the columns past S; any other tile
+                // takes the biased path. Four columns per lane, one warp-wide min and vote
+                // (the loads also bring the bias row into L1 for the biased path; a per-tile
+                // bit from the producer's scan instead was 8% slower on a finite bias).
                 kb = key_bias + static_cast<size_t>(bh / H) * S + kv0;
                 const int c = 4 * static_cast<int>(lane_id());
-                bool zero = true;
+                float bv[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) zero = zero && (c + e >= valid || __ldg(kb + c + e) == 0.f);
-                raw_path = __all_sync(0xffffffffu, zero);
+                for (int e = 0; e < 4; ++e) bv[e] = (c + e < valid) ? __ldg(kb + c + e) : -INFINITY;
+                int first_drop = kTileN;   // this lane's first -inf column
+#pragma unroll
+                for (int e = 3; e >= 0; --e)
+                    if (bv[e] == -INFINITY) first_drop = c + e;
+                const int p = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<uint32_t>(first_drop)));
+                bool prefix = true;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) prefix = prefix && ((c + e < p) ? bv[e] == 0.f : bv[e] == -INFINITY);
+                raw_path = __all_sync(0xffffffffu, prefix);
+                if (raw_path) valid = p;
             }
             uint32_t u[kTileN];
             uint32_t (&ua)[64] = *reinterpret_cast<uint32_t(*)[64]>(u);

@@ -189,19 +189,23 @@ def test_general_finite_key_bias():
     assert_bf16_parity(out, ref, 2, "general key bias")
 
 
+@pytest.mark.parametrize("pattern", ["every_third", "right_padding"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_dropped_keys_weigh_exactly_zero(D):
+def test_dropped_keys_weigh_exactly_zero(D, pattern):
     """Keys dropped by a -inf bias inside tiles that keep other keys: their V rows hold the
     largest finite bf16 value, so any weight above 0 (2^-125 from the polynomial would already
-    give ~7) shows in the output; the result must match the oracle, which drops them."""
+    give ~7) shows in the output; the result must match the oracle, which drops them. Every
+    third key dropped takes the biased path; a right-padded entry (zeros, then -inf) takes the
+    unbiased one with the padding masked."""
     c = syn.encoder_case(2, 3, 600, D, seed=91, softmax_scale=D ** -0.5)
     kb = torch.zeros((2, 600), dtype=torch.float32)
-    kb[:, 1::3] = float("-inf")          # every third key of every tile
-    kb[1, 450:] = float("-inf")          # and a padded tail in entry 1
+    if pattern == "every_third":
+        kb[:, 1::3] = float("-inf")
+    kb[0, 300:] = float("-inf")          # a padded tail in both entries
+    kb[1, 450:] = float("-inf")
     v = c.v.clone()
     big = torch.finfo(torch.bfloat16).max
-    v[:, :, 1::3, :] = big
-    v[1, :, 450:, :] = big
+    v[kb.isinf()[:, None, :, None].expand_as(v)] = big
     case = syn.EncoderCase(c.q, c.k, v, c.softmax_scale, kb)
     out = _run(case)
     assert torch.isfinite(out.float()).all()
