@@ -62,11 +62,15 @@ constexpr int kKOff = kQOff + kTileBytes;
 constexpr int kVOff = kKOff + kStages * kTileBytes;
 constexpr int kBarOff = kVOff + kStages * kTileBytes;
 // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full, s_free, p_ready[4], pv_done,
-// o_final, mma_done, count_ready
+// o_final, mma_done, count_ready, bias_full[S], bias_empty[S]
 constexpr int kPChunks = kTileN / 32;   // P is written, and P.V issued, in 32-key chunks
-constexpr int kNumBars = 1 + 4 * kStages + 6 + kPChunks;
+constexpr int kNumBars = 1 + 4 * kStages + 6 + kPChunks + 2 * kStages;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;   // TMEM address, abort flag, live tile count
-constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+// with a key bias: per ring stage the tile's bias in log2 units (128 floats) and one word,
+// the first -inf column when the tile is a prefix mask (zeros, then -inf), else -1
+constexpr int kBiasOff = (kMiscOff + 16 + 15) & ~15;
+constexpr int kBiasInfoOff = kBiasOff + kStages * kTileN * 4;
+constexpr int kSmemBytes = kBiasInfoOff + kStages * 4 + 1024;
 
 // Key tiles up to the last key whose bias is not -inf (at least one), found by a whole warp:
 // with right padding the trailing tiles hold only -inf keys, which take no part in any row.
@@ -98,6 +102,10 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* o_final = pv_done + 1;
     uint64_t* mma_done = o_final + 1;
     uint64_t* count_ready = mma_done + 1;
+    uint64_t* bias_full = count_ready + 1;      // the producer has staged tile j's bias
+    uint64_t* bias_empty = bias_full + kStages; // the softmax warps are done with it
+    float* bias_s = reinterpret_cast<float*>(smem + kBiasOff);
+    volatile int* bias_info = reinterpret_cast<volatile int*>(smem + kBiasInfoOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 4);
     // with a key bias: the key tiles that hold a kept key (the producer counts them while the
@@ -124,6 +132,10 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(o_final, 1);
         mbar_init(mma_done, 1);
         mbar_init(count_ready, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bias_full[s], 1);
+            mbar_init(&bias_empty[s], 4);   // one arrival per softmax warp
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -167,16 +179,55 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             load_kv(0);
         }
         __syncwarp();
-        int n_kv = n_kv_all;
-        if constexpr (kHasBias) {
-            n_kv = live_key_tiles(key_bias + static_cast<size_t>(bh / H) * S, S);
+        if constexpr (!kHasBias) {
+            if (lane_id() == 0)
+                for (int j = 1; j < n_kv_all && ok; ++j) load_kv(j);
+        } else {
+            const float* kb_row = key_bias + static_cast<size_t>(bh / H) * S;
+            const int n_kv = live_key_tiles(kb_row, S);
             if (lane_id() == 0) {
                 *n_live_slot = n_kv;
                 mbar_arrive(count_ready);   // release: the count is visible to the waiters
             }
+            // Tile j's bias into ring stage j % kStages, whole warp, four columns per lane:
+            // in log2 units (-inf kept, a finite value clamped at -FLT_MAX so that its key
+            // stays), and whether the tile is a prefix mask: zeros up to its first -inf
+            // column, -inf from there on (no bias, or the end of a right-padded entry).
+            auto stage_bias = [&](int j) -> bool {
+                const int st = j % kStages;
+                const uint32_t use = j / kStages;
+                if (use > 0 && !mbar_wait_warp(&bias_empty[st], (use - 1) & 1, abort_flag)) return false;
+                const int c = 4 * static_cast<int>(lane_id());
+                const int valid = S - j * kTileN;
+                float bv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) bv[e] = (c + e < valid) ? __ldg(kb_row + j * kTileN + c + e) : -INFINITY;
+                int first_drop = kTileN;
+#pragma unroll
+                for (int e = 3; e >= 0; --e)
+                    if (bv[e] == -INFINITY) first_drop = c + e;
+                const int p = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<uint32_t>(first_drop)));
+                bool prefix = true;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) prefix = prefix && ((c + e < p) ? bv[e] == 0.f : bv[e] == -INFINITY);
+                prefix = __all_sync(0xffffffffu, prefix);
+                float w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[e] = bv[e] == -INFINITY ? -INFINITY : fmaxf(bv[e] * kLog2e, -FLT_MAX);
+                reinterpret_cast<float4*>(bias_s + st * kTileN)[lane_id()] = make_float4(w[0], w[1], w[2], w[3]);
+                if (lane_id() == 0) bias_info[st] = prefix ? p : -1;
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(&bias_full[st]);   // release: the stage is visible
+                return true;
+            };
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok) ok = stage_bias(0);
+            for (int j = 1; j < n_kv && ok; ++j) {
+                if (lane_id() == 0) load_kv(j);
+                ok = __shfl_sync(0xffffffffu, ok, 0);   // lane 0's copies decide for the warp
+                if (ok) ok = stage_bias(j);
+            }
         }
-        if (lane_id() == 0)
-            for (int j = 1; j < n_kv && ok; ++j) load_kv(j);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -263,29 +314,23 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int kv0 = j * kTileN;
             int valid = S - kv0;    // columns of this tile that take part (the rest are -inf)
             bool raw_path = true;   // scores taken as they are (no key bias on this tile)
-            const float* kb = nullptr;
+            const float* bl = nullptr;
             if constexpr (kHasBias) {
-                // A tile whose bias is 0 on a prefix of its columns and -inf on the rest (no
-                // bias at all, or the end of a right-padded entry) is computed as without a
-                // bias, with the -inf part masked like the columns past S; any other tile
-                // takes the biased path. Four columns per lane, one warp-wide min and vote
-                // (the loads also bring the bias row into L1 for the biased path; a per-tile
-                // bit from the producer's scan instead was 8% slower on a finite bias).
-                kb = key_bias + static_cast<size_t>(bh / H) * S + kv0;
-                const int c = 4 * static_cast<int>(lane_id());
-                float bv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) bv[e] = (c + e < valid) ? __ldg(kb + c + e) : -INFINITY;
-                int first_drop = kTileN;   // this lane's first -inf column
-#pragma unroll
-                for (int e = 3; e >= 0; --e)
-                    if (bv[e] == -INFINITY) first_drop = c + e;
-                const int p = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<uint32_t>(first_drop)));
-                bool prefix = true;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) prefix = prefix && ((c + e < p) ? bv[e] == 0.f : bv[e] == -INFINITY);
-                raw_path = __all_sync(0xffffffffu, prefix);
-                if (raw_path) valid = p;
+                // the producer has staged this tile's bias: a prefix mask (zeros, then -inf)
+                // is computed as without a bias with its -inf part masked like the columns
+                // past S; any other tile adds the staged log2-unit bias to its scores
+                const int stb = j % kStages;
+                ok = mbar_wait_warp(&bias_full[stb], (j / kStages) & 1, abort_flag);
+                if (!ok) break;
+                const int info = bias_info[stb];
+                raw_path = info >= 0;
+                if (raw_path) {
+                    valid = info;
+                    __syncwarp();
+                    if (lane_id() == 0) mbar_arrive(&bias_empty[stb]);
+                } else {
+                    bl = bias_s + stb * kTileN;
+                }
             }
             uint32_t u[kTileN];
             uint32_t (&ua)[64] = *reinterpret_cast<uint32_t(*)[64]>(u);
@@ -341,31 +386,27 @@ encoder_1q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 __syncwarp();
                 if (lane_id() == 0) mbar_arrive(s_free);
                 pv_seen = j == 0 || mbar_test(pv_done, (j - 1) & 1);
-                // biased score of column i in log2 units (scale folded in); -inf where the
-                // bias is -inf or past S; a finite bias stays finite (a -FLT_MAX fill keeps its
-                // key). Every lane reads the same biases: 16-byte broadcast loads.
+                // biased score in log2 units: one FMA per score against the staged bias
+                // (-inf where the key is dropped or past S: the staged value is -inf there)
                 mx[0] = mx[1] = mx[2] = mx[3] = -INFINITY;
 #pragma unroll
                 for (int i = 0; i < kTileN; i += 4) {
-                    float4 b4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-                    if (i + 3 < valid && ((reinterpret_cast<uintptr_t>(kb + i) & 15u) == 0)) {
-                        b4 = __ldg(reinterpret_cast<const float4*>(kb + i));
-                    } else {
-                        if (i < valid) b4.x = __ldg(kb + i);
-                        if (i + 1 < valid) b4.y = __ldg(kb + i + 1);
-                        if (i + 2 < valid) b4.z = __ldg(kb + i + 2);
-                        if (i + 3 < valid) b4.w = __ldg(kb + i + 3);
-                    }
-                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x = bb[e] == -INFINITY
-                                            ? -INFINITY
-                                            : fmaf(__uint_as_float(u[i + e]), scale_log2, fmaxf(bb[e] * kLog2e, -FLT_MAX));
-                        u[i + e] = __float_as_uint(x);
-                        mx[e] = fmaxf(mx[e], x);
-                    }
+                    const float4 b4 = *reinterpret_cast<const float4*>(bl + i);
+                    const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
+                                                  make_float2(scale_log2, scale_log2), make_float2(b4.x, b4.y));
+                    const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(u[i + 2]), __uint_as_float(u[i + 3])),
+                                                  make_float2(scale_log2, scale_log2), make_float2(b4.z, b4.w));
+                    u[i] = __float_as_uint(x01.x);
+                    u[i + 1] = __float_as_uint(x01.y);
+                    u[i + 2] = __float_as_uint(x23.x);
+                    u[i + 3] = __float_as_uint(x23.y);
+                    mx[0] = fmaxf(mx[0], x01.x);
+                    mx[1] = fmaxf(mx[1], x01.y);
+                    mx[2] = fmaxf(mx[2], x23.x);
+                    mx[3] = fmaxf(mx[3], x23.y);
                 }
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(&bias_empty[j % kStages]);
                 m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             }
             // log2-unit factor of the scores in u: the scale on the raw path, 1 on the biased one
