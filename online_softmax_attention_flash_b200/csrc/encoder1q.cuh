@@ -3,13 +3,14 @@
 //
 // What it computes: the same as encoder_fwd_kernel (encoder.cuh), at D = 64: out[b,h] =
 // softmax(scale * Q K^T + key_bias[b]) V, q/k/v/out [B, H, S, 64] bf16, key_bias [B, S] fp32
-// additive or none. With a key bias (kHasBias) the producer counts the key tiles up to the
-// entry's last kept key while the first copies fly (the tiles after it are never loaded);
-// a tile whose bias is 0 on a prefix of its columns and -inf on the rest (no bias, or the
-// end of a right-padded entry) takes the unbiased path with the -inf part masked, any other
-// tile turns its scores into biased log2-unit scores before the max, and a dropped key (bias
-// -inf) weighs exactly 0 wherever the polynomial would give 2^-125, since its V row may hold
-// any finite value.
+// additive or none. With a key bias (kHasBias) the producer warp counts the key tiles up to
+// the entry's last kept key while the first copies fly (the tiles after it are never
+// loaded), and stages each live tile's bias in log2 units in a shared-memory ring beside the
+// K / V stages, with a word that says whether the tile is a prefix mask (0 on its first
+// columns, -inf on the rest: no bias, or the end of a right-padded entry). A prefix-mask tile
+// takes the unbiased path with the -inf part masked; any other tile adds the staged bias to
+// its scores (one FMA per score) before the max. A dropped key (bias -inf) weighs exactly 0
+// wherever the polynomial would give 2^-125, since its V row may hold any finite value.
 //
 // How. A CTA owns 128 query rows of one (b, h) and streams the key sequence in 128-key
 // tiles through a 2-stage TMA ring: warp 5 (one thread) issues QK(j+1) as soon as the
