@@ -17,8 +17,9 @@
 // softmax has read S(j), and PV(j) in four 32-key parts, each as soon as the softmax warps
 // have written that chunk of P(j) (one completion commit per tile: a commit per part costs
 // more than the finer waits it would allow); warps 0-3 are the softmax, one thread per row
-// holding all 128 scores of its row, so the row max needs no exchange between warps. TMEM holds S (128 columns), O (64) and P (64, bf16 pairs): 256 columns,
-// and the CTA needs ~81 KB of shared memory, so two CTAs share an SM. The two query tiles
+// holding all 128 scores of its row, so the row max needs no exchange between warps. TMEM
+// holds S (128 columns), O (64) and P (64, bf16 pairs): 256 columns, and the CTA needs
+// ~82 KB of shared memory, so two CTAs share an SM. The two query tiles
 // an SM works on then belong to different CTAs: nothing in the issue order couples their
 // phases, and one CTA's exponentials (MUFU) overlap the other's max, stores and waits.
 // The running max may be stale by up to 2^8 (the final O / l uses the same reference);
