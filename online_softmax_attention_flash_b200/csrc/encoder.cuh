@@ -64,11 +64,17 @@ struct Cfg {
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
     // o_final, xchg[2] (row-max / row-sum exchange between the two halves of a tile),
-    // count_ready (the number of key tiles with a kept key is known; key-bias kernels)
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 1;
+    // count_ready (the number of key tiles with a kept key is known; key-bias kernels),
+    // bias_full[S] / bias_empty[S] (a key tile's bias staged by the producer / read by every
+    // softmax warp; key-bias kernels)
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 2 + 1 + 2 * kStages;
     static constexpr int kXchgOff = kBarOff + kNumBars * 8;   // float [2 buf][2 tile][2 half][128]
-    static constexpr int kMiscOff = kXchgOff + 2 * 2 * 2 * 128 * 4;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + tmem slot, abort flag, alignment slack
+    static constexpr int kMiscOff = kXchgOff + 2 * 2 * 2 * 128 * 4;   // tmem slot, abort flag, count
+    // key-bias kernels: per ring stage the tile's bias in log2 units (128 floats) and one word,
+    // the first -inf column when the tile is a prefix mask (zeros, then -inf), else -1
+    static constexpr int kBiasOff = (kMiscOff + 16 + 15) & ~15;   // 16-byte stores
+    static constexpr int kBiasInfoOff = kBiasOff + kStages * kTileN * 4;
+    static constexpr int kSmemBytes = kBiasInfoOff + kStages * 4 + 1024;   // + alignment slack
     // TMEM columns: S_t at 128 t, O_t at 256 + D t. TMEM is full, so P_t (bf16 pairs) is
     // written over the first 64 columns of S_t.
     static constexpr uint32_t kColS0 = 0;
@@ -86,6 +92,8 @@ struct Bars {
     uint64_t* o_final;
     uint64_t* xchg;
     uint64_t* count_ready;
+    uint64_t* bias_full;
+    uint64_t* bias_empty;
 };
 
 template <int D>
@@ -103,6 +111,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
     r.o_final = r.p_ready + 2;
     r.xchg = r.o_final + 1;
     r.count_ready = r.xchg + 2;
+    r.bias_full = r.count_ready + 1;
+    r.bias_empty = r.bias_full + C::kStages;
     return r;
 }
 
@@ -136,6 +146,8 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // with a key bias: the key tiles that hold a kept key (the producer counts them while the
     // first copies are in flight and publishes the count here)
     volatile int* n_live_slot = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
+    float* bias_s = reinterpret_cast<float*>(smem + C::kBiasOff);
+    volatile int* bias_info = reinterpret_cast<volatile int*>(smem + C::kBiasInfoOff);
 
     if (threadIdx.x == 0) {
         mbar_init(bars.q_full, 1);
@@ -152,6 +164,10 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         mbar_init(bars.o_final, 1);
         mbar_init(bars.count_ready, 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&bars.bias_full[s], 1);
+            mbar_init(&bars.bias_empty[s], kSoftmaxWarps);   // every softmax warp reads it
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -203,16 +219,53 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             load_kv(0);
         }
         __syncwarp();
-        int n_kv = n_kv_all;
         if constexpr (kHasBias) {
-            n_kv = live_key_tiles(key_bias + static_cast<size_t>(bh / H) * S, S);
+            const float* kb_row = key_bias + static_cast<size_t>(bh / H) * S;
+            const int n_kv = live_key_tiles(kb_row, S);
             if (lane_id() == 0) {
                 *n_live_slot = n_kv;
                 mbar_arrive(bars.count_ready);   // release: the count is visible to the waiters
             }
-        }
-        if (lane_id() == 0) {
-            for (int j = 1; j < n_kv && ok; ++j) load_kv(j);
+            // Tile j's bias into ring stage j % kStages, whole warp, four columns per lane:
+            // in log2 units (-inf kept, a finite value clamped at -FLT_MAX so that its key
+            // stays), and whether the tile is a prefix mask: zeros up to its first -inf
+            // column, -inf from there on (no bias, or the end of a right-padded entry).
+            auto stage_bias = [&](int j) -> bool {
+                const int st = j % C::kStages;
+                const uint32_t use = j / C::kStages;
+                if (use > 0 && !mbar_wait_warp(&bars.bias_empty[st], (use - 1) & 1, abort_flag)) return false;
+                const int c = 4 * static_cast<int>(lane_id());
+                const int valid = S - j * kTileN;
+                float bv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) bv[e] = (c + e < valid) ? __ldg(kb_row + j * kTileN + c + e) : -INFINITY;
+                int first_drop = kTileN;
+#pragma unroll
+                for (int e = 3; e >= 0; --e)
+                    if (bv[e] == -INFINITY) first_drop = c + e;
+                const int p = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<uint32_t>(first_drop)));
+                bool prefix = true;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) prefix = prefix && ((c + e < p) ? bv[e] == 0.f : bv[e] == -INFINITY);
+                prefix = __all_sync(0xffffffffu, prefix);
+                float w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[e] = bv[e] == -INFINITY ? -INFINITY : fmaxf(bv[e] * kLog2e, -FLT_MAX);
+                reinterpret_cast<float4*>(bias_s + st * kTileN)[lane_id()] = make_float4(w[0], w[1], w[2], w[3]);
+                if (lane_id() == 0) bias_info[st] = prefix ? p : -1;
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(&bars.bias_full[st]);   // release: the stage is visible
+                return true;
+            };
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok) ok = stage_bias(0);
+            for (int j = 1; j < n_kv && ok; ++j) {
+                if (lane_id() == 0) load_kv(j);
+                ok = __shfl_sync(0xffffffffu, ok, 0);   // lane 0's copies decide for the warp
+                if (ok) ok = stage_bias(j);
+            }
+        } else if (lane_id() == 0) {
+            for (int j = 1; j < n_kv_all && ok; ++j) load_kv(j);
             // on an abort (here or in another role) the copies are drained at teardown
         }
         __syncwarp();
@@ -314,7 +367,6 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t tOh = tmem_base + lane_off + C::kColO0 + t * D + hf * (D / 2);
         float* xchg = reinterpret_cast<float*>(smem + C::kXchgOff);
         auto xslot = [&](int buf, int half) { return xchg + ((buf * 2 + t) * 2 + half) * kTileM + r; };
-        const int b = bh / H;
         const int col0 = hf * kHalf;
         float m_run = -INFINITY;   // running max, log2 units (scale folded in)
         float l_run = 0.f;         // running sum over this warp's half of the columns
@@ -342,26 +394,34 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (!ok) break;
             tc_fence_after();
             const int kv0 = j * kTileN;
-            const int valid = S - kv0;   // keys of this tile that exist
-            const float* kb = nullptr;
-            bool bias_zero = true;
+            int valid = S - kv0;   // keys of this tile that take part (the rest are -inf)
+            bool raw_path = true;
+            const float* bl = nullptr;
             if constexpr (kHasBias) {
-                kb = key_bias + static_cast<size_t>(b) * S + kv0;
-                // A tile whose bias values (of this warp's half, columns before S) are all zero
-                // is computed exactly as without a bias (the common case of right padding: only
-                // the tiles past a sequence's length carry -inf).
-                const int c = col0 + 2 * static_cast<int>(lane_id());
-                const bool zero = (c >= valid || __ldg(kb + c) == 0.f) &&
-                                  (c + 1 >= valid || __ldg(kb + c + 1) == 0.f);
-                bias_zero = __all_sync(0xffffffffu, zero);
+                // the producer has staged this tile's bias: a prefix mask (zeros, then -inf: no
+                // bias, or the end of a right-padded entry) is computed as without a bias with
+                // its -inf part masked like the columns past S; any other tile adds the staged
+                // log2-unit bias to its scores
+                const int stb = j % C::kStages;
+                ok = mbar_wait_warp(&bars.bias_full[stb], (j / C::kStages) & 1, abort_flag);
+                if (!ok) break;
+                const int info = bias_info[stb];
+                raw_path = info >= 0;
+                if (raw_path) {
+                    valid = info;
+                    __syncwarp();
+                    if (lane_id() == 0) mbar_arrive(&bars.bias_empty[stb]);
+                } else {
+                    bl = bias_s + stb * kTileN + col0;
+                }
             }
             uint32_t u[kHalf];
             tmem_ld64_wait(tSh, u);
-            // A ragged last tile without a key bias keeps the raw-score path: the columns
-            // past S become -inf (the scale is positive, so the max is unchanged); their
-            // weights are 0, or 2^-125 where the polynomial takes them, against V rows that
-            // the copy zero-filled.
-            const bool raw_path = !kHasBias || bias_zero;
+            // On the raw-score path the columns past S (or past a prefix mask's end) become
+            // -inf (the scale is positive, so the max is unchanged); their weights are 0, or
+            // 2^-125 where the polynomial takes them against V rows that the copy zero-filled
+            // (the key-bias build makes those weights exactly 0: a dropped key's V row may hold
+            // any finite value).
             if (raw_path && valid < kTileN) {
 #pragma unroll
                 for (int i = 0; i < kHalf; ++i)
@@ -384,32 +444,27 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 m_half = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * scale_log2;
             } else if constexpr (kHasBias) {
-                // key bias on this tile: score of column i in log2 units (scale folded in),
-                // -inf where masked; finite biases stay finite (a -FLT_MAX fill keeps its key).
-                // Every lane reads the same biases: 16-byte broadcast loads, 4 columns each.
-#pragma unroll
-                for (int i = 0; i < kHalf; i += 4) {
-                    float4 b4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-                    if (col0 + i + 3 < valid && ((reinterpret_cast<uintptr_t>(kb + col0 + i) & 15u) == 0)) {
-                        b4 = __ldg(reinterpret_cast<const float4*>(kb + col0 + i));
-                    } else {
-                        if (col0 + i < valid) b4.x = __ldg(kb + col0 + i);
-                        if (col0 + i + 1 < valid) b4.y = __ldg(kb + col0 + i + 1);
-                        if (col0 + i + 2 < valid) b4.z = __ldg(kb + col0 + i + 2);
-                        if (col0 + i + 3 < valid) b4.w = __ldg(kb + col0 + i + 3);
-                    }
-                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float sv = __uint_as_float(u[i + e]);
-                        u[i + e] = __float_as_uint(bb[e] == -INFINITY
-                                                       ? -INFINITY
-                                                       : fmaf(sv, scale_log2, fmaxf(bb[e] * kLog2e, -FLT_MAX)));
-                    }
-                }
+                // biased score in log2 units: one packed FMA per two scores against the staged
+                // bias (-inf where the key is dropped or past S: the staged value is -inf there)
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(u[i]));
+                for (int i = 0; i < kHalf; i += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(bl + i);
+                    const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
+                                                  make_float2(scale_log2, scale_log2), make_float2(b4.x, b4.y));
+                    const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(u[i + 2]), __uint_as_float(u[i + 3])),
+                                                  make_float2(scale_log2, scale_log2), make_float2(b4.z, b4.w));
+                    u[i] = __float_as_uint(x01.x);
+                    u[i + 1] = __float_as_uint(x01.y);
+                    u[i + 2] = __float_as_uint(x23.x);
+                    u[i + 3] = __float_as_uint(x23.y);
+                    mx[0] = fmaxf(mx[0], x01.x);
+                    mx[1] = fmaxf(mx[1], x01.y);
+                    mx[2] = fmaxf(mx[2], x23.x);
+                    mx[3] = fmaxf(mx[3], x23.y);
+                }
+                __syncwarp();
+                if (lane_id() == 0) mbar_arrive(&bars.bias_empty[j % C::kStages]);
                 m_half = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             }
             float m_other;
@@ -433,10 +488,15 @@ encoder_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (raw_path) {
                         const float2 x = __ffma2_rn(sv, make_float2(scale_log2, scale_log2),
                                                     make_float2(-m_use, -m_use));
-                        // the polynomial also takes the -inf columns past S of a ragged tile:
-                        // it clamps them to 2^-125, and their V rows are zero-filled
-                        if ((kk & 7) < kPolyEighths) pv = exp2_poly2(x);
-                        else pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        if ((kk & 7) < kPolyEighths) {
+                            pv = exp2_poly2(x);
+                            if constexpr (kHasBias) {   // a dropped key weighs exactly 0
+                                if (x.x == -INFINITY) pv.x = 0.f;
+                                if (x.y == -INFINITY) pv.y = 0.f;
+                            }
+                        } else {
+                            pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        }
                     } else {
                         pv = make_float2(ex2_approx(sv.x - m_use), ex2_approx(sv.y - m_use));
                     }
