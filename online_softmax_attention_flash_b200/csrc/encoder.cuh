@@ -22,8 +22,12 @@
 //     is exact); one column pair in eight takes 2^x from an FMA-pipe polynomial
 //     instead of the MUFU unit;
 //   * warp 16 (one elected thread) is the TMA producer; with a key bias the whole warp
-//     also counts the key tiles up to the batch entry's last kept key, and the tiles
-//     after it (right padding) are neither loaded nor computed.
+//     also counts the key tiles up to the batch entry's last kept key (the tiles after it
+//     are neither loaded nor computed) and stages each live tile's bias in log2 units in a
+//     shared-memory ring, with a word that says whether the tile is a prefix mask (0 on
+//     its first columns, -inf on the rest): such a tile runs the unbiased path with the
+//     -inf part masked, any other adds the staged bias to its scores (one FMA per score),
+//     and a dropped key weighs exactly 0 (its V row may hold any finite value).
 // The two query tiles ping-pong: while one warpgroup computes exponentials the
 // tensor core runs the other tile's MMAs.
 #pragma once
